@@ -1,0 +1,235 @@
+/*
+ * cql.h -- C ABI of libcql, the B200 (sm_100a) compressed linear layer.
+ *
+ * The layer computes, for activations x [B][K] and outputs y [B][N],
+ *
+ *     y = deq(Q (.) M) x  +  S_csr x  +  deq(L_q) (deq(R_q) x)
+ *
+ * where Q holds low-bit codes of W (symmetric clipped int4/int3 with one fp16
+ * scale per 128 columns, as in SLiM-Quant; or a 3/4-bit per-row non-uniform
+ * table, as in SqueezeLLM), M is a 2:4 or unstructured-50% sparsity mask,
+ * S_csr an optional fp16 CSR matrix of outliers (SqueezeLLM's dense-and-sparse
+ * split), and L_q, R_q rank-r adapters quantised AbsMax int4 in groups of 128
+ * (SLiM's "Low-rank adapter quantization").
+ *
+ * Sources: "SLiM: One-shot Quantization and Sparsity with Low-rank
+ * Approximation for LLM Weight Compression" (review summary: SLIM-Quant,
+ * Low-rank adapter quantization; rebuttal: Unstructured vs. 2:4 Sparsity,
+ * Speedup Comparison without LoRA) and "SqueezeLLM: Dense-and-Sparse
+ * Quantization" (Approach; Key results).  The pages fix no API, byte layout,
+ * scale dtype, rounding or tie rule; those are defined here.
+ *
+ * Conventions for every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller, except the
+ *     descriptor/layout/output-scalar pointers, which are host pointers.
+ *   - The library allocates no memory and keeps no global state.  Scratch
+ *     memory comes from the caller's workspace.
+ *   - Calls are stream-ordered and asynchronous.  Argument and format errors
+ *     are returned synchronously before anything is launched.  Errors found
+ *     on the device (a bad header, a bounded wait that ran out) are written to
+ *     the error word at the start of the workspace; read it with
+ *     cql_get_device_status.
+ *   - Nothing crosses the ABI as an exception; the library never exits,
+ *     aborts or traps.
+ *
+ * ------------------------------------------------------------------------
+ * PACKED FORMAT (version 1)
+ * ------------------------------------------------------------------------
+ * A packed weight is one contiguous device buffer: a 512-byte header followed
+ * by up to 11 planes, in the order of the CQL_PLANE_* indices.  Every plane
+ * starts on a 256-byte boundary; an absent plane has length 0 and the offset
+ * where it would start.  All multi-byte fields are little-endian.
+ *
+ * Header: "CQL1", uint32 version = 1, cql_desc (64 bytes), then the
+ * cql_layout (uint64 total_bytes, uint64 nnz, uint64 off[12], uint64 len[12]);
+ * the rest of the 512 bytes is zero.
+ *
+ * Row-interleaved planes (VALUES, META, SCALES, VOFF, R_VALUES, R_SCALES,
+ * L_VALUES).  Each row contributes row_bytes bytes (a multiple of 16, zero
+ * padded).  Rows are grouped in blocks of 32; a block is stored as a run of
+ * 512-byte slabs, slab s holding bytes [16s, 16s+16) of each of its 32 rows in
+ * row order.  Byte j of row i is at
+ *     ((i / 32) * (row_bytes / 16) + j / 16) * 512 + (i % 32) * 16 + (j % 16).
+ * (32 consecutive lanes reading 16 bytes each read one slab: one coalesced
+ * 512-byte access per warp.)
+ *
+ * Bit streams.  Code c of a row occupies stream bits [b*c, b*c + b) for b-bit
+ * codes; stream bit t is bit (t % 8) of row byte t / 8.
+ *
+ * VALUES  b-bit codes of the kept entries of each row, in column order.
+ *         int4/int3: u = q + 2^(b-1), q in [-(2^(b-1)-1), 2^(b-1)-1].
+ *         lut3/lut4: index of the row's centroid.
+ *         kept per row = K/2 under 2:4 and bitmap50, K without a mask.
+ *         row_bytes = pad16(ceil(kept * b / 8)).
+ * META    2:4: 4-bit pattern index p of column group g (columns 4g..4g+3) at
+ *         stream bits [4g, 4g+4); p names the kept pair (i0, i1), i0 < i1, in
+ *         lexicographic order: 0:(0,1) 1:(0,2) 2:(0,3) 3:(1,2) 4:(1,3) 5:(2,3).
+ *         bitmap50: bit k of the row stream is 1 when column k is kept.
+ *         row_bytes = K/8.  Absent without a mask.
+ * SCALES  int4/int3: fp16 scale of columns [128g, 128g+128) at row bytes
+ *         [2g, 2g+2); row_bytes = pad16(K/64).
+ *         lut3/lut4: the row's 2^b fp16 centroids; row_bytes = 2^(b+1).
+ * VOFF    bitmap50 only: uint16 index, in the row's VALUES stream, of the
+ *         first kept code of columns [128g, ...) at row bytes [2g, 2g+2);
+ *         row_bytes = pad16(K/64).  (Lets a reader start mid-row.)
+ * CSR_ROWPTR  int32 [N+1]      present when outlier_frac > 0
+ * CSR_COL     uint16 [nnz]     columns ascending within a row
+ * CSR_VAL     fp16 [nnz]       value = fp16(w - dense part at that entry)
+ * R_VALUES  int4 codes u = q + 8 of R [r][K]; rows padded to a multiple of 32
+ *           (padding rows all zero bytes, zero scales); row_bytes = K/2.
+ * R_SCALES  fp16 scale of R row j, columns [128g, 128g+128); row_bytes =
+ *           pad16(K/64).
+ * L_VALUES  int4 codes u = q + 8 of L [N][r]; row_bytes = pad16(r/2).
+ * L_SCALES  fp16 [N/128][r], plain row-major: scale of column j over rows
+ *           [128g, 128g+128) at index g*r + j.
+ *
+ * Encoding rules (shared by pack_compressed_weight and the CPU oracle; every
+ * real-valued step is evaluated in fp64 from exact widenings, then rounded to
+ * fp16 round-to-nearest-even, ties in selections go to the lower index):
+ *   1. outliers: the floor(f*N*K) entries of largest |w| over the whole matrix;
+ *   2. mask on |w|: 2:4 keeps the two largest of every 4 columns; bitmap50
+ *      keeps the K/2 largest of every row;
+ *   3. int codecs: s = fp16((alpha * amax) / qmax) with amax over the group's
+ *      non-outlier entries, q = clamp(rint(w / s), -qmax, qmax), q = 0 when
+ *      s = 0; qmax = 7 (int4) or 3 (int3);
+ *      lut codecs: centroid j = linear-interpolated quantile of the row's
+ *      sorted non-outlier values at p = (j + 1/2)/2^b, rounded to fp16; every
+ *      entry takes the nearest centroid;
+ *   4. CSR values as above;
+ *   5. adapters: s = fp16(amax / 7), q = clamp(rint(v / s), -7, 7), groups of
+ *      128 along K for R and along N for L.
+ */
+#ifndef CQL_H
+#define CQL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CQL_VERSION 1
+#define CQL_HEADER_BYTES 512
+#define CQL_NPLANES 12
+#define CQL_GROUP 128
+#define CQL_MAX_DECODE_BATCH 16
+
+typedef enum {
+  CQL_OK = 0,
+  CQL_ERR_ARG = 1,          /* null pointer, bad enum, bad size relation    */
+  CQL_ERR_ALIGN = 2,        /* pointer not aligned as documented            */
+  CQL_ERR_FORMAT = 3,       /* header magic/version/descriptor mismatch     */
+  CQL_ERR_SIZE = 4,         /* buffer or workspace too small                */
+  CQL_ERR_UNSUPPORTED = 5,  /* valid but not implemented combination        */
+  CQL_ERR_CUDA = 6,         /* a CUDA runtime call failed                   */
+  CQL_ERR_TIMEOUT = 7       /* a bounded device wait ran out                */
+} cql_status;
+
+typedef enum { CQL_MASK_NONE = 0, CQL_MASK_2_4 = 1, CQL_MASK_BITMAP50 = 2 } cql_mask;
+typedef enum {
+  CQL_CODEC_INT4_SYM = 0, CQL_CODEC_INT3_SYM = 1, CQL_CODEC_LUT3_ROW = 2, CQL_CODEC_LUT4_ROW = 3
+} cql_codec;
+typedef enum { CQL_DT_F32 = 0, CQL_DT_F16 = 1, CQL_DT_BF16 = 2 } cql_dtype;
+
+enum {
+  CQL_PLANE_HEADER = 0, CQL_PLANE_VALUES = 1, CQL_PLANE_META = 2, CQL_PLANE_SCALES = 3,
+  CQL_PLANE_VOFF = 4, CQL_PLANE_CSR_ROWPTR = 5, CQL_PLANE_CSR_COL = 6, CQL_PLANE_CSR_VAL = 7,
+  CQL_PLANE_R_VALUES = 8, CQL_PLANE_R_SCALES = 9, CQL_PLANE_L_VALUES = 10, CQL_PLANE_L_SCALES = 11
+};
+
+/* Term toggles (cql_desc.flags, read by compressed_linear_forward only; used
+ * by the per-term parity tests). */
+#define CQL_FLAG_NO_MAIN 0x1u
+#define CQL_FLAG_NO_CSR 0x2u
+#define CQL_FLAG_NO_LOWRANK 0x4u
+
+/* Layer descriptor, 64 bytes, stored verbatim in the packed header. */
+typedef struct cql_desc {
+  int32_t n_out;          /* N, rows of W; multiple of 128, <= 2^20          */
+  int32_t k_in;           /* K, columns of W; multiple of 128, <= 65536      */
+  int32_t mask;           /* cql_mask                                        */
+  int32_t codec;          /* cql_codec; lut codecs need CQL_MASK_NONE        */
+  int32_t group;          /* weight scale group; must be 128                 */
+  float clip_alpha;       /* SLiM-Quant clip alpha in (0, 1]                 */
+  float outlier_frac;     /* CSR fraction f in [0, 1/16]; 0 = no CSR         */
+  int32_t rank;           /* adapter rank r, multiple of 16, <= 256; 0 = none */
+  int32_t adapter_bits;   /* must be 4                                       */
+  int32_t adapter_group;  /* must be 128                                     */
+  uint32_t flags;         /* CQL_FLAG_* term toggles                         */
+  int32_t reserved[5];    /* zero                                            */
+} cql_desc;
+
+typedef struct cql_layout {
+  uint64_t total_bytes;   /* size of the packed buffer                       */
+  uint64_t nnz;           /* CSR entries, floor(f * N * K)                   */
+  uint64_t off[CQL_NPLANES];
+  uint64_t len[CQL_NPLANES];
+} cql_layout;
+
+typedef struct CUstream_st* cql_stream_t;   /* == cudaStream_t */
+
+/* Human-readable name of a status code.  Never returns NULL. */
+const char* cql_status_string(cql_status s);
+
+/* Library version (CQL_VERSION) and the packed-format version it writes. */
+int32_t cql_version(void);
+
+/* Validate a descriptor and compute the packed layout.  Host only: touches no
+ * GPU.  Returns CQL_ERR_ARG / CQL_ERR_UNSUPPORTED for descriptors the library
+ * cannot pack. */
+cql_status cql_packed_layout(const cql_desc* desc, cql_layout* out);
+
+/* Scratch bytes pack_compressed_weight needs.  Host only. */
+cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
+
+/* Encode W (and the adapters) into the packed format (rules above).
+ *   W         device, [N][K] row-major, w_dt = CQL_DT_F32 or CQL_DT_BF16,
+ *             16-byte aligned.
+ *   L         device fp32 [N][r] row-major, or NULL when rank == 0.
+ *   R         device fp32 [r][K] row-major, or NULL when rank == 0.
+ *   packed    device, >= cql_layout.total_bytes, 256-byte aligned; every byte
+ *             of it is written.
+ *   workspace device scratch of >= cql_pack_workspace_size bytes, 256-byte
+ *             aligned; its contents on entry do not matter.
+ * The result is bit-exact with the CPU oracle on every byte.  Inputs must be
+ * finite. */
+cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt,
+                                  const float* L, const float* R, void* packed,
+                                  uint64_t packed_bytes, void* workspace, uint64_t ws_bytes,
+                                  cql_stream_t stream);
+
+/* Workspace bytes compressed_linear_forward needs for this layer and batch.
+ * Host only. */
+cql_status cql_workspace_size(const cql_desc* desc, int32_t batch, uint64_t* bytes);
+
+/* Zero a forward workspace (required once before its first use; the forward
+ * leaves the parts it reuses zeroed again when it completes). */
+cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t stream);
+
+/* y = deq(Q (.) M) x + S_csr x + deq(L_q)(deq(R_q) x)  for a packed layer.
+ *   desc      host copy of the descriptor the layer was packed with (its
+ *             flags select the terms computed).
+ *   packed    device, the packed buffer, 256-byte aligned.
+ *   x         device [batch][K], x_dt = CQL_DT_F16 or CQL_DT_BF16, 16-byte
+ *             aligned.
+ *   y         device [batch][N], y_dt = CQL_DT_F32, F16 or BF16, 16-byte
+ *             aligned; fp32 accumulation, one final round to y_dt.
+ *   batch     1..16 runs the CUDA-core decode GEMV (bandwidth bound); larger
+ *             batches run the tcgen05 tensor-core prefill GEMM, which is
+ *             implemented for 2:4 int4 layers (others: CQL_ERR_UNSUPPORTED).
+ *   workspace device, >= cql_workspace_size bytes, 256-byte aligned, zeroed
+ *             once by cql_workspace_init.  Calls sharing one workspace must
+ *             be ordered on one stream.
+ */
+cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, const void* x,
+                                     cql_dtype x_dt, void* y, cql_dtype y_dt, int32_t batch,
+                                     void* workspace, uint64_t ws_bytes, cql_stream_t stream);
+
+/* Wait for the stream, then read and clear the device error word of a
+ * workspace: *out = CQL_OK or the cql_status a kernel recorded. */
+cql_status cql_get_device_status(void* workspace, cql_stream_t stream, cql_status* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CQL_H */

@@ -1,0 +1,397 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks an oracle function against brute force on tiny inputs, a
+closed form, an invariant the method guarantees, or an independent library
+routine -- chosen so that a plausible slip (a dropped term, a wrong sign or
+index, a transposed operand, a wrong tie rule) fails at least one of them.
+CPU only.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+from workloads import make_layer_inputs, workload
+
+RNG = np.random.default_rng(1234)
+
+
+# ---------------------------------------------------------------------------
+# independent helpers (exact rational arithmetic, pure Python)
+# ---------------------------------------------------------------------------
+
+def fp16_round_exact(v: Fraction) -> Fraction:
+    """Round a rational to the nearest binary16 value, ties to even, by exact
+    arithmetic (normal and subnormal ranges; no overflow in these tests)."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = math.floor(math.log2(a))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -14)                      # subnormals share the exponent -14
+    ulp = Fraction(2) ** (e - 10)
+    m = a / ulp
+    fl = math.floor(m)
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * ulp
+
+
+def half_ulp16(v: float) -> float:
+    a = abs(v)
+    if a == 0:
+        return 2.0 ** -25
+    e = max(math.floor(math.log2(a)), -14)
+    return 2.0 ** (e - 11)
+
+
+# ---------------------------------------------------------------------------
+# fp16 rounding
+# ---------------------------------------------------------------------------
+
+def test_fp16_round_ties_and_single_rounding():
+    one = 1.0
+    # exact tie between 1 and 1 + 2^-10 rounds to the even significand (1.0)
+    assert O.fp16_round(one + 2.0 ** -11)[()] == 1.0
+    # tie between 1 + 2^-10 (odd) and 1 + 2^-9 (even) rounds up
+    assert O.fp16_round(one + 3 * 2.0 ** -11)[()] == one + 2.0 ** -9
+    # just above a tie: a double rounding through fp32 would give 1.0
+    assert O.fp16_round(one + 2.0 ** -11 + 2.0 ** -40)[()] == one + 2.0 ** -10
+    # random values agree with exact rational rounding
+    vals = RNG.standard_normal(2000) * 10.0 ** RNG.uniform(-6, 3, 2000)
+    got = O.fp16_round(vals)
+    for v, g in zip(vals, got):
+        assert Fraction(g) == fp16_round_exact(Fraction(v))
+
+
+# ---------------------------------------------------------------------------
+# outliers
+# ---------------------------------------------------------------------------
+
+def test_outlier_count_closed_form():
+    d = O.OracleDesc(4096, 4096, O.MASK_NONE, O.CODEC_LUT3, outlier_frac=0.0045)
+    # 0.0045 * 4096^2 = 75497.472 -> floor
+    assert O.n_outliers(d) == 75497
+    d0 = O.OracleDesc(4096, 4096, O.MASK_NONE, O.CODEC_LUT3, outlier_frac=0.0)
+    assert O.n_outliers(d0) == 0
+
+
+def test_select_outliers_brute_force_with_ties():
+    w = RNG.standard_normal((6, 8)).round(1)          # many equal magnitudes
+    w[2, 3] = -w[0, 1]                                 # explicit tie of |w|
+    for cnt in (0, 1, 5, 13, 48):
+        flat = [(abs(float(v)), i) for i, v in enumerate(w.reshape(-1))]
+        chosen = sorted(i for _, i in sorted(flat, key=lambda t: (-t[0], t[1]))[:cnt])
+        assert list(O.select_outliers(w, cnt)) == chosen
+
+
+def test_outlier_threshold_invariant():
+    w = RNG.standard_t(4, size=(64, 128)) * 0.02
+    idx = O.select_outliers(w, 37)
+    a = np.abs(w).reshape(-1)
+    inside = np.zeros(a.size, bool)
+    inside[idx] = True
+    assert inside.sum() == 37
+    assert a[inside].min() >= a[~inside].max()
+
+
+# ---------------------------------------------------------------------------
+# masks
+# ---------------------------------------------------------------------------
+
+def _best_pair_brute(vals):
+    """The 2:4 pair of largest summed |w|, the lexicographically first on a tie:
+    equal to keeping the top 2 magnitudes with ties to the lower index."""
+    best, best_p = None, None
+    for p, (i0, i1) in enumerate(O.PAIRS_2OF4):
+        s = abs(vals[i0]) + abs(vals[i1])
+        if best is None or s > best:
+            best, best_p = s, p
+    return best_p
+
+
+def test_mask_2of4_brute_force():
+    # integer-valued weights produce plenty of ties
+    w = RNG.integers(-3, 4, size=(16, 64)).astype(np.float64)
+    keep, pat = O.mask_2of4(w)
+    for n in range(w.shape[0]):
+        for g in range(w.shape[1] // 4):
+            vals = [float(v) for v in w[n, 4 * g: 4 * g + 4]]
+            p = _best_pair_brute(vals)
+            assert pat[n, g] == p
+            i0, i1 = O.PAIRS_2OF4[p]
+            exp = [i in (i0, i1) for i in range(4)]
+            assert list(keep[n, 4 * g: 4 * g + 4]) == exp
+
+
+def test_mask_2of4_invariants():
+    w = RNG.standard_normal((32, 256))
+    keep, pat = O.mask_2of4(w)
+    assert (keep.reshape(32, 64, 4).sum(-1) == 2).all()
+    a = np.abs(w).reshape(32, 64, 4)
+    kk = keep.reshape(32, 64, 4)
+    assert (np.where(kk, a, np.inf).min(-1) >= np.where(kk, -np.inf, a).max(-1)).all()
+    # an already 2:4 sparse matrix keeps its own pattern
+    w2 = np.where(keep, w, 0.0)
+    keep2, pat2 = O.mask_2of4(w2)
+    assert (keep2 == keep).all() and (pat2 == pat).all()
+
+
+def test_mask_bitmap50_invariants_and_ties():
+    w = RNG.standard_normal((8, 256))
+    keep = O.mask_bitmap50(w)
+    assert (keep.sum(1) == 128).all()
+    a = np.abs(w)
+    for n in range(8):
+        assert a[n, keep[n]].min() >= a[n, ~keep[n]].max()
+    # all-equal magnitudes: the lower half of the columns is kept
+    w3 = np.tile(np.array([1.0, -1.0]), (2, 64))
+    k3 = O.mask_bitmap50(w3)
+    assert k3[:, :64].all() and not k3[:, 64:].any()
+
+
+# ---------------------------------------------------------------------------
+# uniform codec
+# ---------------------------------------------------------------------------
+
+def test_uniform_scale_exact_rational():
+    """s = fp16(alpha * amax / qmax) against exact rational arithmetic."""
+    for bits in (4, 3):
+        qmax = 2 ** (bits - 1) - 1
+        w = RNG.standard_normal((4, 512)) * 0.02
+        q, s = O.quantize_uniform(w, bits, 0.9)
+        alpha = Fraction(float(np.float32(0.9)))
+        for n in range(4):
+            for g in range(4):
+                amax = max(abs(Fraction(float(v))) for v in w[n, 128 * g: 128 * g + 128])
+                assert Fraction(float(s[n, g])) == fp16_round_exact(alpha * amax / qmax)
+
+
+def test_uniform_codes_on_grid_and_error_bound():
+    w = RNG.standard_normal((8, 256)) * 0.02
+    w[3, 17] = 0.9                                  # a clipped outlier
+    for bits in (4, 3):
+        qmax = 2 ** (bits - 1) - 1
+        q, s = O.quantize_uniform(w, bits, 0.9)
+        assert q.min() >= -qmax and q.max() <= qmax
+        sb = np.repeat(s, 128, axis=1)
+        what = q * sb
+        inside = np.abs(w) <= qmax * sb
+        assert (np.abs(w - what)[inside] <= sb[inside] / 2).all()
+        # clipped values sit at the grid edge with the right sign
+        out = ~inside
+        assert (q[out] == np.sign(w[out]) * qmax).all()
+
+
+def test_uniform_textbook_rtn_special_case():
+    """alpha = 1: the element of largest |w| of a group maps to +-qmax, and
+    re-quantising the dequantised matrix reproduces the codes (idempotence)."""
+    w = RNG.standard_normal((4, 384)) * 0.05
+    q, s = O.quantize_uniform(w, 4, 1.0)
+    for n in range(4):
+        for g in range(3):
+            seg = w[n, 128 * g: 128 * g + 128]
+            j = int(np.argmax(np.abs(seg)))
+            assert abs(int(q[n, 128 * g + j])) == 7
+    what = q * np.repeat(s, 128, axis=1)
+    q2, s2 = O.quantize_uniform(what, 4, 1.0)
+    assert (q2 == q).all()
+
+
+def test_uniform_zero_group():
+    w = np.zeros((1, 256))
+    w[0, 200] = 0.3
+    q, s = O.quantize_uniform(w, 4, 0.9)
+    assert s[0, 0] == 0 and (q[0, :128] == 0).all()
+    assert q[0, 200] == 7
+
+
+def test_uniform_rounding_half_even():
+    """A value exactly halfway between two grid points rounds to the even code."""
+    s = 2.0 ** -6                                    # exact in fp16
+    w = np.zeros((1, 128))
+    w[0, 0] = 7 * s                                  # amax; alpha 1 -> scale s
+    w[0, 1] = 2.5 * s
+    w[0, 2] = -1.5 * s
+    w[0, 3] = 0.5 * s
+    q, sc = O.quantize_uniform(w, 4, 1.0)
+    assert sc[0, 0] == s
+    assert list(q[0, :4]) == [7, 2, -2, 0]
+
+
+# ---------------------------------------------------------------------------
+# LUT codec
+# ---------------------------------------------------------------------------
+
+def test_lut_centroids_match_numpy_quantile():
+    w = RNG.standard_t(4, size=(16, 512)) * 0.02
+    for bits in (3, 4):
+        c = O.lut_centroids(w, bits)
+        p = (np.arange(2 ** bits) + 0.5) / 2 ** bits
+        for n in range(16):
+            ref = np.quantile(w[n].astype(np.float64), p, method="linear")
+            assert (c[n] == O.fp16_round(ref)).all()
+
+
+def test_lut_centroids_exclude_outliers():
+    w = RNG.standard_normal((4, 256))
+    ex = np.zeros_like(w, dtype=bool)
+    ex[1, [3, 100, 200]] = True
+    c = O.lut_centroids(w, 3, exclude=ex)
+    p = (np.arange(8) + 0.5) / 8
+    ref = np.quantile(w[1][~ex[1]], p, method="linear")
+    assert (c[1] == O.fp16_round(ref)).all()
+
+
+def test_lut_assign_brute_force():
+    w = RNG.standard_normal((5, 64)) * 0.02
+    c = O.lut_centroids(w, 3)
+    c[2, 4] = c[2, 3]                                # duplicate centroid: tie
+    code = O.lut_assign(w, c)
+    for n in range(5):
+        for kk in range(64):
+            d = [abs(float(w[n, kk]) - float(c[n, j])) for j in range(8)]
+            assert code[n, kk] == d.index(min(d))
+
+
+# ---------------------------------------------------------------------------
+# adapters
+# ---------------------------------------------------------------------------
+
+def test_adapter_groups_run_along_model_dimension():
+    R = RNG.standard_normal((16, 512)) * 0.01
+    L = RNG.standard_normal((256, 16)) * 0.01
+    rq, rs = O.quantize_adapter_rows(R)
+    lq, ls = O.quantize_adapter_cols(L)
+    assert rs.shape == (16, 4) and ls.shape == (2, 16)
+    for j in range(16):
+        for g in range(4):
+            seg = R[j, 128 * g: 128 * g + 128]
+            amax = np.abs(seg).max()
+            assert Fraction(float(rs[j, g])) == fp16_round_exact(Fraction(float(amax)) / 7)
+            assert abs(int(rq[j, 128 * g + int(np.argmax(np.abs(seg)))])) == 7
+        for g in range(2):
+            seg = L[128 * g: 128 * g + 128, j]
+            assert Fraction(float(ls[g, j])) == fp16_round_exact(Fraction(float(np.abs(seg).max())) / 7)
+    assert np.abs(rq).max() <= 7 and np.abs(lq).max() <= 7
+
+
+# ---------------------------------------------------------------------------
+# CSR
+# ---------------------------------------------------------------------------
+
+def test_csr_sums_back_to_outliers():
+    wl = workload("lut_dense_sparse", n=128, k=256, seed=77)
+    inp = make_layer_inputs(wl)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"])
+    rp, col, val = parts["csr_row_ptr"], parts["csr_col"], parts["csr_val"]
+    assert rp[-1] == math.floor(float(np.float32(0.0045)) * 128 * 256) == len(val)
+    w = inp["w"].astype(np.float64)
+    dense = parts["w_dense"]
+    rows = np.repeat(np.arange(128), np.diff(rp))
+    for r_, c_, v_ in zip(rows, col, val):
+        resid = w[r_, c_] - dense[r_, c_]
+        assert abs(v_ - resid) <= half_ulp16(v_)
+    # columns ascending within each row
+    for n in range(128):
+        seg = col[rp[n]: rp[n + 1]]
+        assert (np.diff(seg) > 0).all()
+    # outliers hold the largest magnitudes
+    a = np.abs(w)
+    inside = np.zeros_like(a, dtype=bool)
+    inside[rows, col] = True
+    assert a[inside].min() >= a[~inside].max()
+
+
+# ---------------------------------------------------------------------------
+# forward pass
+# ---------------------------------------------------------------------------
+
+def _brute_forward(parts, desc, x):
+    """y by explicit loops over every weight, rebuilding W_hat element by
+    element from codes, scales, mask, CSR and adapters."""
+    n, k, r = desc.n_out, desc.k_in, desc.rank
+    W = [[0.0] * k for _ in range(n)]
+    keep = parts["keep"]
+    for i in range(n):
+        for j in range(k):
+            if not keep[i, j]:
+                continue
+            if desc.codec in (O.CODEC_INT4, O.CODEC_INT3):
+                W[i][j] = float(parts["q"][i, j]) * float(parts["scales"][i, j // 128])
+            else:
+                W[i][j] = float(parts["centroids"][i, parts["codes"][i, j]])
+    if "csr_row_ptr" in parts:
+        rp = parts["csr_row_ptr"]
+        for i in range(n):
+            for e in range(rp[i], rp[i + 1]):
+                W[i][int(parts["csr_col"][e])] += float(parts["csr_val"][e])
+    if r:
+        for i in range(n):
+            for j in range(k):
+                acc = 0.0
+                for t in range(r):
+                    lv = float(parts["L_q"][i, t]) * float(parts["L_s"][i // 128, t])
+                    rv = float(parts["R_q"][t, j]) * float(parts["R_s"][t, j // 128])
+                    acc += lv * rv
+                W[i][j] += acc
+    y = np.zeros((x.shape[0], n))
+    for b in range(x.shape[0]):
+        for i in range(n):
+            y[b, i] = math.fsum(W[i][j] * float(x[b, j]) for j in range(k))
+    return y
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict(n=128, k=256, rank=16)),
+    ("down_unstructured", dict(n=128, k=256, rank=32, codec="int3")),
+    ("lut_dense_sparse", dict(n=128, k=256)),
+])
+def test_forward_matches_brute_force(name, over):
+    wl = workload(name, **over)
+    inp = make_layer_inputs(wl, max_batch=2)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"])
+    y = O.forward(parts, inp["x"])
+    yb = _brute_forward(parts, d, inp["x"])
+    assert O.rel_err(y, yb) < 1e-12
+
+
+def test_forward_linear_and_term_isolation():
+    wl = workload("tiny", n=128, k=256, rank=16)
+    inp = make_layer_inputs(wl, max_batch=3)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"])
+    x = inp["x"].astype(np.float64)
+    y1 = O.forward(parts, x[:1])
+    y2 = O.forward(parts, x[1:2])
+    y12 = O.forward(parts, x[:1] + 2.0 * x[1:2])
+    assert O.rel_err(y12, y1 + 2.0 * y2) < 1e-12
+    # a zero quantised part leaves exactly the adapter term
+    p0 = dict(parts)
+    p0["w_dense"] = np.zeros_like(parts["w_dense"])
+    lr = O.forward(p0, x)
+    exp = (x @ parts["R_hat"].T) @ parts["L_hat"].T
+    assert O.rel_err(lr, exp) < 1e-12
+    # rank 0: no adapter term
+    d0 = O.desc_for(workload("tiny", n=128, k=256, rank=0))
+    parts0 = O.compress(d0, inp["w"])
+    assert "R_hat" not in parts0
+    m, c, l = O.forward_terms(parts0, x)
+    assert not l.any() and not c.any()
+
+
+def test_rel_err_metric():
+    ref = np.array([[1.0, -2.0, 0.0, 1e-9]])
+    rms = math.sqrt((1 + 4 + 0 + 1e-18) / 4)
+    y = ref + np.array([[0.0, 0.004, 1e-3, 0.0]])
+    assert abs(O.rel_err(y, ref) - max(0.004 / 2.0, 1e-3 / rms)) < 1e-15
