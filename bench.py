@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed linear layer forward pass on B200.
+
+One step = one pass of the whole decode hot path over one batch:
+    y = deq(Q (.) M) x + S_csr x + deq(L_q) (deq(R_q) x)
+for the LLaMA-7B MLP up/gate projection (11008 x 4096, bf16 weights, 2:4
+mask, int4 group-128 clipped codes, rank-128 int4 adapters, batch 1), packed
+once on the GPU by the library and then run through its C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cql|reference]
+
+Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs and
+bracketed by a barrier + synchronize, timed with CUDA events on the launching
+stream; max over ranks.  Inputs rotate over enough copies of the packed
+weights to exceed 2x L2, so every step reads its weights from HBM.  Under
+torchrun each rank runs the same layer on its own GPU (independent replicas,
+weak scaling, no data-path collective).
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (the
+plain fp64 definition) on the host cores on bounded row samples of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode GEMV effective HBM GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=("cql", "reference"), default="cql")
+    ap.add_argument("--workload", default="mlp_up")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary per-workload lines")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-oracle sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+PLANE_HEADER, PLANE_VOFF = 0, 4          # include/cql.h CQL_PLANE_HEADER / CQL_PLANE_VOFF
+
+
+def algorithmic_bytes(layout, batch, n, k, x_bytes=2, y_bytes=2):
+    """Bytes the layer must move per call: every packed plane except the header
+    and the VOFF index (a format aid), plus x and y."""
+    planes = sum(int(layout.len[i]) for i in range(12) if i not in (PLANE_HEADER, PLANE_VOFF))
+    return planes + batch * k * x_bytes + batch * n * y_bytes
+
+
+def desc_from_workload(C, wl):
+    mask = {"2:4": C.CQL_MASK_2_4, "bitmap50": C.CQL_MASK_BITMAP50, "none": C.CQL_MASK_NONE}[wl.mask]
+    codec = {"int4": C.CQL_CODEC_INT4_SYM, "int3": C.CQL_CODEC_INT3_SYM, "lut3": C.CQL_CODEC_LUT3_ROW,
+             "lut4": C.CQL_CODEC_LUT4_ROW}[wl.codec]
+    return C.make_desc(wl.n, wl.k, mask, codec, wl.clip_alpha, wl.outlier_frac, wl.rank)
+
+
+def device_inputs(torch, inp, wl, dev):
+    """Seeded inputs to the device, in the dtypes the workload delivers them in."""
+    if wl.w_dtype == "bf16":
+        W = torch.from_numpy(inp["w_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+    else:
+        W = torch.from_numpy(inp["w"]).to(dev)
+    L = torch.from_numpy(inp["L"]).to(dev) if inp["L"] is not None else None
+    R = torch.from_numpy(inp["R"]).to(dev) if inp["R"] is not None else None
+    xt = torch.float16 if wl.x_dtype == "f16" else torch.bfloat16
+    x = torch.from_numpy(inp["x_bits"].view(np.int16)).to(dev).view(xt)
+    return W, L, R, x
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "sparse_quantized_rank_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    decode sources changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", f"{name}.md")
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"```json\s*(\{.*?\})\s*```", open(p).read(), re.S)
+    if not m:
+        return None
+    d = json.loads(m.group(1))
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_rate(wl, batch, seconds, steps=None, warmup=0):
+    """Time the oracle's fp64 forward on row samples on the host cores.
+    Returns (GB/s of algorithmic bytes, steps, rows per step, threads)."""
+    import oracle as O
+    from workloads import make_layer_inputs
+    inp = make_layer_inputs(wl, max_batch=batch)
+    od = O.desc_for(wl)
+    parts = O.compress(od, inp["w"], inp["L"], inp["R"])
+    lay = O.packed_layout(od)
+    x = inp["x"][:batch].astype(np.float64)
+    planes = sum(lay["len"][i] for i in range(12) if i not in (O.P_HEADER, O.P_VOFF))
+    per_row = planes / wl.n
+    t0 = time.perf_counter()
+    O.forward(parts, x, rows=np.arange(min(wl.n, 256)))
+    t_row = max((time.perf_counter() - t0) / min(wl.n, 256), 1e-7)
+    if steps is None:
+        rows = min(wl.n, max(32, int(0.5 / t_row)))
+        steps = max(1, int(seconds / (t_row * rows)))
+    else:
+        rows = min(wl.n, max(32, int(seconds / max(steps + warmup, 1) / t_row)))
+    rng = np.random.default_rng(0)
+    for _ in range(warmup):
+        O.forward(parts, x, rows=np.sort(rng.choice(wl.n, rows, replace=False)))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.forward(parts, x, rows=np.sort(rng.choice(wl.n, rows, replace=False)))
+    dt = time.perf_counter() - t0
+    nbytes = steps * (rows * per_row + batch * wl.k * 2 + batch * rows * 2)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    return nbytes / dt / 1e9, steps, rows, threads, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from workloads import workload
+    wl = workload(args.workload)
+    gbs, steps, rows, threads, dt = cpu_oracle_rate(wl, args.batch, seconds=60.0, steps=args.steps,
+                                                    warmup=args.warmup)
+    sample = f"{rows} of {wl.n} output rows per step (fp64 oracle forward), {steps} steps"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": dt / max(steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl_name(wl, args.batch)},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def wl_name(wl, batch):
+    return (f"{wl.name} {wl.n}x{wl.k} {wl.mask} {wl.codec} g128"
+            + (f" r{wl.rank}" if wl.rank else "") + (f" csr{wl.outlier_frac}" if wl.outlier_frac else "")
+            + f" batch {batch}")
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Bench:
+    """One packed layer, rotated over enough copies to defeat L2."""
+
+    def __init__(self, wl, batch, dev, torch, C):
+        from workloads import make_layer_inputs
+        self.torch, self.C, self.wl, self.batch = torch, C, wl, batch
+        inp = make_layer_inputs(wl, max_batch=batch)
+        W, L, R, x = device_inputs(torch, inp, wl, dev)
+        self.desc = desc_from_workload(C, wl)
+        self.layer = C.CompressedLinear(self.desc, W, L, R)
+        del W, L, R
+        torch.cuda.synchronize()
+        self.layout = self.layer.layout
+        l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20)
+        self.ncopy = max(2, math.ceil(2.2 * l2 / self.layout.total_bytes))
+        self.copies = [self.layer.packed] + [self.layer.packed.clone() for _ in range(self.ncopy - 1)]
+        self.x = x[:batch].contiguous()
+        self.xdt = C._dt_of(self.x)
+        self.y = torch.empty(batch, wl.n, dtype=self.x.dtype, device=dev)
+        self.ws, self.wsb = self.layer.workspace(batch)
+        self.bytes = algorithmic_bytes(self.layout, batch, wl.n, wl.k)
+        self.kernels_per_step = 2 if wl.rank else 1
+
+    def step(self, i, stream):
+        C = self.C
+        C.compressed_linear_forward(self.desc, self.copies[i % self.ncopy], self.x, self.xdt, self.y, self.xdt,
+                                    self.batch, self.ws, self.wsb, stream)
+
+    def timed(self, steps, warmup, stream, sampler=None, barrier=None):
+        """(total seconds for `steps` steps, mean seconds per step from events
+        inside the graph)."""
+        torch = self.torch
+        for i in range(warmup):
+            self.step(i, stream.cuda_stream)
+        g_steps = min(steps, 1000)
+        n_rep, rem = divmod(steps, g_steps)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(g_steps)]
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            s = torch.cuda.current_stream().cuda_stream
+            for i in range(g_steps):
+                ev[i][0].record()
+                self.step(i, s)
+                ev[i][1].record()
+        graph_rem = None
+        if rem:
+            graph_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_rem, stream=stream):
+                s = torch.cuda.current_stream().cuda_stream
+                for i in range(rem):
+                    self.step(i, s)
+        graph.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if barrier:
+            barrier()
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.start()
+            time.sleep(0.3)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(n_rep):
+                graph.replay()
+            if graph_rem is not None:
+                graph_rem.replay()
+            end.record(stream)
+        end.synchronize()
+        torch.cuda.synchronize()
+        clocks = sampler.stop() if sampler else None
+        if barrier:
+            barrier()
+        total = start.elapsed_time(end) / 1e3
+        per = float(np.mean([a.elapsed_time(b) for a, b in ev])) / 1e3
+        del graph, graph_rem
+        return total, per, clocks
+
+    def e2e(self, steps, stream):
+        """Same metric through the public API with host buffers: H2D of x and
+        D2H of y inside every step."""
+        torch = self.torch
+        xh = self.x.cpu().pin_memory()
+        yh = torch.empty(self.y.shape, dtype=self.y.dtype).pin_memory()
+        xd = torch.empty_like(self.x)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(20):
+                xd.copy_(xh, non_blocking=True)
+                self.layer.forward(xd, out=self.y, stream=stream)
+                yh.copy_(self.y, non_blocking=True)
+            stream.synchronize()
+            start.record(stream)
+            for i in range(steps):
+                xd.copy_(xh, non_blocking=True)
+                self.C.compressed_linear_forward(self.desc, self.copies[i % self.ncopy], xd, self.xdt, self.y,
+                                                 self.xdt, self.batch, self.ws, self.wsb, stream.cuda_stream)
+                yh.copy_(self.y, non_blocking=True)
+            end.record(stream)
+        end.synchronize()
+        dt = start.elapsed_time(end) / 1e3
+        return self.bytes * steps / dt / 1e9, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+
+
+def run_cql(args):
+    import torch
+    import torch.distributed as dist
+    import sparse_quantized_rank_b200 as C
+    from workloads import workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = workload(args.workload)
+    b = Bench(wl, args.batch, dev, torch, C)
+    stream = torch.cuda.Stream(device=dev)
+    sampler = ClockSampler(local)
+    total, per_step, clocks = b.timed(args.steps, max(args.warmup, 3), stream, sampler, barrier)
+    if world > 1:
+        t = torch.tensor([total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    value = world * b.bytes * args.steps / total / 1e9
+    e2e_gbs, h2d, d2h = b.e2e(min(args.steps, 2000), stream)
+    peak, peak_src = measured_peaks()
+    achieved = b.bytes / per_step / 1e9
+    prof_name = f"decode_{wl.name}_b{args.batch}"
+    traffic = profiled_traffic(prof_name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl_name(wl, args.batch), "bytes_per_step": b.bytes,
+                   "l2": f"inputs larger than L2: {b.ncopy} rotating packed copies "
+                         f"({b.ncopy * b.layout.total_bytes / 1e6:.0f} MB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_8TBs": value / world / 8000.0 * 100,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6650 GB/s",
+                     "kernel": "k_decode (2:4 int4) + k_lowrank_stage1 overlapped by PDL; per-step event time"},
+        "e2e": {"value": e2e_gbs * world, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "public API per step: H2D x, forward, D2H y; no graph, host launch cost included"},
+        "gpu_launches": args.steps * b.kernels_per_step,
+        "clocks": clocks,
+    }
+    del b
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1:
+        gbs, steps, rows, threads, dt = cpu_oracle_rate(wl, args.batch, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"fp64 oracle forward over {rows} of {wl.n} rows, {steps} steps, "
+                                          f"{dt:.1f} s"}
+    if not args.no_extra:
+        line["extra"] = extra_lines(torch, C, dev, stream, barrier)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def extra_lines(torch, C, dev, stream, barrier):
+    """Secondary decode measurements (same method, shorter runs)."""
+    from workloads import workload
+    out = []
+    peak, _ = measured_peaks()
+    for name, batch in (("tiny", 1), ("mlp_up", 4), ("mlp_up", 16), ("lut_dense_sparse", 1),
+                        ("lut_dense_sparse", 8), ("down_unstructured", 1), ("down_unstructured", 16)):
+        wl = workload(name)
+        b = Bench(wl, batch, dev, torch, C)
+        total, per, _ = b.timed(20000, 200, stream)
+        gbs = b.bytes * 20000 / total / 1e9
+        out.append({"workload": wl_name(wl, batch), "GB/s": round(gbs, 1), "us_per_step": round(total / 20000 * 1e6, 3),
+                    "us_per_step_events": round(per * 1e6, 3), "frac_of_measured_hbm": round(gbs / peak, 4),
+                    "bytes_per_step": b.bytes})
+        del b
+        torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cql(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -226,7 +226,8 @@ def lut_centroids(w: np.ndarray, bits: int, exclude: Optional[np.ndarray] = None
     the row's non-outlier values at p_j = (j + 1/2) / 2^bits,
         h = (n_r - 1) p_j,  c_j = v[floor h] + (h - floor h)(v[floor h + 1] - v[floor h])
     with v the sorted values, evaluated in fp64 in exactly that order, then
-    rounded to fp16.  A row with no values gets all-zero centroids.
+    rounded to fp16.  A zero centroid is +0 (the sign of a zero from a sort
+    is not defined).  A row with no values gets all-zero centroids.
     Returns fp64 [N][2^bits] holding fp16 values."""
     w = np.asarray(w, dtype=np.float64)
     n, k = w.shape
@@ -246,7 +247,7 @@ def lut_centroids(w: np.ndarray, bits: int, exclude: Optional[np.ndarray] = None
         vlo = v[rows, lo]
         vhi = v[rows, hi]
         c = vlo + frac * (vhi - vlo)
-        out[:, j] = np.where(nr > 0, c, 0.0)
+        out[:, j] = np.where(nr > 0, c, 0.0) + 0.0      # -0 -> +0
     return fp16_round(out)
 
 

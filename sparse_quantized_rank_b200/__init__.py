@@ -1,0 +1,231 @@
+"""Python binding of libcql, the B200 compressed linear layer.
+
+    y = deq(Q (.) M) x + S_csr x + deq(L_q) (deq(R_q) x)
+
+Argument marshalling only: every function below calls the C ABI declared in
+``include/cql.h`` with the same name, passing device pointers taken from torch
+tensors (torch supplies device memory and streams, nothing else).  There is no
+CPU fallback: if ``libcql.so`` is missing or cannot be loaded, the first call
+raises.
+
+``CompressedLinear`` is a small convenience owner of the packed buffer and
+workspace for one layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcql.so")
+
+# enums (include/cql.h)
+CQL_OK, CQL_ERR_ARG, CQL_ERR_ALIGN, CQL_ERR_FORMAT, CQL_ERR_SIZE, CQL_ERR_UNSUPPORTED, \
+    CQL_ERR_CUDA, CQL_ERR_TIMEOUT = range(8)
+CQL_MASK_NONE, CQL_MASK_2_4, CQL_MASK_BITMAP50 = 0, 1, 2
+CQL_CODEC_INT4_SYM, CQL_CODEC_INT3_SYM, CQL_CODEC_LUT3_ROW, CQL_CODEC_LUT4_ROW = 0, 1, 2, 3
+CQL_DT_F32, CQL_DT_F16, CQL_DT_BF16 = 0, 1, 2
+CQL_FLAG_NO_MAIN, CQL_FLAG_NO_CSR, CQL_FLAG_NO_LOWRANK = 1, 2, 4
+CQL_NPLANES = 12
+CQL_MAX_DECODE_BATCH = 16
+
+EXPORTED = (
+    "cql_status_string", "cql_version", "cql_packed_layout", "cql_pack_workspace_size",
+    "pack_compressed_weight", "cql_workspace_size", "cql_workspace_init",
+    "compressed_linear_forward", "cql_get_device_status",
+)
+
+
+class cql_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_out", ctypes.c_int32), ("k_in", ctypes.c_int32), ("mask", ctypes.c_int32),
+        ("codec", ctypes.c_int32), ("group", ctypes.c_int32), ("clip_alpha", ctypes.c_float),
+        ("outlier_frac", ctypes.c_float), ("rank", ctypes.c_int32), ("adapter_bits", ctypes.c_int32),
+        ("adapter_group", ctypes.c_int32), ("flags", ctypes.c_uint32), ("reserved", ctypes.c_int32 * 5),
+    ]
+
+
+class cql_layout(ctypes.Structure):
+    _fields_ = [
+        ("total_bytes", ctypes.c_uint64), ("nnz", ctypes.c_uint64),
+        ("off", ctypes.c_uint64 * CQL_NPLANES), ("len", ctypes.c_uint64 * CQL_NPLANES),
+    ]
+
+
+class CqlError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {cql_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libcql.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_quantized_rank_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, U64, I32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int32
+        L.cql_status_string.restype = ctypes.c_char_p
+        L.cql_status_string.argtypes = [ctypes.c_int]
+        L.cql_version.restype = I32
+        L.cql_packed_layout.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(cql_layout)]
+        L.cql_pack_workspace_size.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(U64)]
+        L.pack_compressed_weight.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, U64, P, U64, P]
+        L.cql_workspace_size.argtypes = [ctypes.POINTER(cql_desc), I32, ctypes.POINTER(U64)]
+        L.cql_workspace_init.argtypes = [P, U64, P]
+        L.compressed_linear_forward.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P, ctypes.c_int,
+                                                I32, P, U64, P]
+        L.cql_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+        for fn in EXPORTED[2:]:
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != CQL_OK:
+        raise CqlError(st, where)
+
+
+def make_desc(n_out: int, k_in: int, mask: int = CQL_MASK_2_4, codec: int = CQL_CODEC_INT4_SYM,
+              clip_alpha: float = 0.9, outlier_frac: float = 0.0, rank: int = 0, flags: int = 0) -> cql_desc:
+    d = cql_desc()
+    d.n_out, d.k_in, d.mask, d.codec, d.group = n_out, k_in, mask, codec, 128
+    d.clip_alpha, d.outlier_frac, d.rank = clip_alpha, outlier_frac, rank
+    d.adapter_bits, d.adapter_group, d.flags = 4, 128, flags
+    return d
+
+
+# ---------------------------------------------------------------------------
+# the C ABI, same names
+# ---------------------------------------------------------------------------
+
+def cql_status_string(s: int) -> str:
+    return lib().cql_status_string(int(s)).decode()
+
+
+def cql_version() -> int:
+    return int(lib().cql_version())
+
+
+def cql_packed_layout(desc: cql_desc) -> cql_layout:
+    out = cql_layout()
+    _check(lib().cql_packed_layout(ctypes.byref(desc), ctypes.byref(out)), "cql_packed_layout")
+    return out
+
+
+def cql_pack_workspace_size(desc: cql_desc) -> int:
+    v = ctypes.c_uint64()
+    _check(lib().cql_pack_workspace_size(ctypes.byref(desc), ctypes.byref(v)), "cql_pack_workspace_size")
+    return int(v.value)
+
+
+def pack_compressed_weight(desc, W, w_dt, L, R, packed, packed_bytes, workspace, ws_bytes, stream=None):
+    _check(lib().pack_compressed_weight(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(L), _ptr(R), _ptr(packed),
+                                        int(packed_bytes), _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "pack_compressed_weight")
+
+
+def cql_workspace_size(desc: cql_desc, batch: int) -> int:
+    v = ctypes.c_uint64()
+    _check(lib().cql_workspace_size(ctypes.byref(desc), int(batch), ctypes.byref(v)), "cql_workspace_size")
+    return int(v.value)
+
+
+def cql_workspace_init(workspace, ws_bytes, stream=None):
+    _check(lib().cql_workspace_init(_ptr(workspace), int(ws_bytes), _stream(stream)), "cql_workspace_init")
+
+
+def compressed_linear_forward(desc, packed, x, x_dt, y, y_dt, batch, workspace, ws_bytes, stream=None):
+    _check(lib().compressed_linear_forward(ctypes.byref(desc), _ptr(packed), _ptr(x), int(x_dt), _ptr(y), int(y_dt),
+                                           int(batch), _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "compressed_linear_forward")
+
+
+def cql_get_device_status(workspace, stream=None) -> int:
+    v = ctypes.c_int()
+    _check(lib().cql_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(v)), "cql_get_device_status")
+    return int(v.value)
+
+
+# ---------------------------------------------------------------------------
+# convenience owner of one packed layer
+# ---------------------------------------------------------------------------
+
+def _dt_of(t) -> int:
+    import torch
+    return {torch.float32: CQL_DT_F32, torch.float16: CQL_DT_F16, torch.bfloat16: CQL_DT_BF16}[t.dtype]
+
+
+class CompressedLinear:
+    """Packs one layer on the GPU and runs its forward pass.
+
+    ``W`` is a CUDA tensor [N][K] (fp32 or bf16), ``L`` [N][r] and ``R`` [r][K]
+    fp32 CUDA tensors (or None when rank is 0).  Buffers are torch tensors
+    allocated once; forward calls allocate only the output tensor (or write
+    into ``out``)."""
+
+    def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None):
+        import torch
+        self.desc = desc
+        self.layout = cql_packed_layout(desc)
+        dev = W.device
+        self.packed = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=dev)
+        pw = cql_pack_workspace_size(desc)
+        pws = torch.empty(max(pw, 256), dtype=torch.uint8, device=dev)
+        pack_compressed_weight(desc, W.contiguous(), _dt_of(W), None if L is None else L.contiguous(),
+                               None if R is None else R.contiguous(), self.packed, self.layout.total_bytes,
+                               pws, pw, stream)
+        self._pack_ws = pws            # kept alive until the pack kernels ran
+        self._ws = {}
+
+    def workspace(self, batch: int, stream=None):
+        import torch
+        nbytes = cql_workspace_size(self.desc, batch)
+        ws = self._ws.get(batch)
+        if ws is None:
+            ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.packed.device)
+            cql_workspace_init(ws, nbytes, stream)
+            self._ws[batch] = ws
+        return ws, nbytes
+
+    def forward(self, x, out_dtype=None, out=None, flags: Optional[int] = None, stream=None):
+        import torch
+        assert x.dim() == 2 and x.shape[1] == self.desc.k_in and x.is_contiguous()
+        batch = x.shape[0]
+        if out is None:
+            out = torch.empty(batch, self.desc.n_out, dtype=out_dtype or x.dtype, device=x.device)
+        ws, nbytes = self.workspace(batch, stream)
+        d = self.desc
+        if flags is not None:
+            d = cql_desc.from_buffer_copy(self.desc)
+            d.flags = flags
+        compressed_linear_forward(d, self.packed, x, _dt_of(x), out, _dt_of(out), batch, ws, nbytes, stream)
+        return out
+
+    def device_status(self, batch: int, stream=None) -> int:
+        ws, _ = self.workspace(batch, stream)
+        return cql_get_device_status(ws, stream)

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* libcql.so loads and exports every function include/cql.h declares;
+* the host layout computation agrees with the oracle's independent one;
+* argument, alignment and size errors come back before anything launches.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+import sparse_quantized_rank_b200 as C
+from sparse_quantized_rank_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return C.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "cql.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\*?\s+\**([a-z_0-9]+)\s*\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert set(names) == set(C.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert C.cql_version() == 1
+    assert C.cql_status_string(C.CQL_ERR_SIZE).startswith("CQL_ERR_SIZE")
+
+
+def test_desc_struct_size():
+    assert ctypes.sizeof(C.cql_desc) == 64
+    assert ctypes.sizeof(C.cql_layout) == 16 + 2 * 8 * 12
+
+
+DESCS = [
+    dict(n_out=256, k_in=512, mask=1, codec=0, rank=16),
+    dict(n_out=11008, k_in=4096, mask=1, codec=0, rank=128),
+    dict(n_out=4096, k_in=4096, mask=0, codec=2, outlier_frac=0.0045),
+    dict(n_out=4096, k_in=11008, mask=2, codec=1, rank=64),
+    dict(n_out=128, k_in=384, mask=1, codec=1, rank=48),
+    dict(n_out=384, k_in=256, mask=0, codec=3, outlier_frac=0.01, rank=32),
+    dict(n_out=128, k_in=128, mask=2, codec=0, outlier_frac=0.001),
+]
+
+
+@pytest.mark.parametrize("kw", DESCS)
+def test_layout_matches_oracle(lib, kw):
+    d = C.make_desc(**kw)
+    lay = C.cql_packed_layout(d)
+    od = O.OracleDesc(kw["n_out"], kw["k_in"], kw["mask"], kw["codec"], 0.9, kw.get("outlier_frac", 0.0),
+                      kw.get("rank", 0))
+    ol = O.packed_layout(od)
+    assert list(lay.off) == ol["off"]
+    assert list(lay.len) == ol["len"]
+    assert lay.total_bytes == ol["total"] and lay.nnz == ol["nnz"]
+
+
+def test_descriptor_validation(lib):
+    ok = dict(n_out=256, k_in=512, mask=1, codec=0, rank=16)
+    C.cql_packed_layout(C.make_desc(**ok))
+    bad = [
+        (dict(ok, n_out=200), C.CQL_ERR_ARG),
+        (dict(ok, k_in=100), C.CQL_ERR_ARG),
+        (dict(ok, mask=3), C.CQL_ERR_ARG),
+        (dict(ok, codec=7), C.CQL_ERR_ARG),
+        (dict(ok, rank=8), C.CQL_ERR_ARG),
+        (dict(ok, rank=512), C.CQL_ERR_ARG),
+        (dict(ok, clip_alpha=0.0), C.CQL_ERR_ARG),
+        (dict(ok, clip_alpha=1.5), C.CQL_ERR_ARG),
+        (dict(ok, outlier_frac=-0.1), C.CQL_ERR_ARG),
+        (dict(ok, codec=2), C.CQL_ERR_UNSUPPORTED),          # LUT needs no mask
+        (dict(ok, mask=0, codec=2, k_in=32768), C.CQL_ERR_UNSUPPORTED),
+    ]
+    for kw, st in bad:
+        with pytest.raises(C.CqlError) as ei:
+            C.cql_packed_layout(C.make_desc(**kw))
+        assert ei.value.status == st, kw
+    d = C.make_desc(**ok)
+    d.group = 64
+    with pytest.raises(C.CqlError) as ei:
+        C.cql_packed_layout(d)
+    assert ei.value.status == C.CQL_ERR_UNSUPPORTED
+
+
+def test_call_errors_return_before_launch(lib):
+    """Null, misaligned and undersized arguments are rejected on the host."""
+    d = C.make_desc(256, 512, rank=16)
+    lay = C.cql_packed_layout(d)
+    ws = C.cql_workspace_size(d, 1)
+    fake = 1 << 40                                  # never dereferenced
+    L = lib
+    st = L.compressed_linear_forward(ctypes.byref(d), None, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 1, fake, ws, None)
+    assert st == C.CQL_ERR_ARG
+    st = L.compressed_linear_forward(ctypes.byref(d), fake + 16, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 1, fake, ws,
+                                     None)
+    assert st == C.CQL_ERR_ALIGN
+    st = L.compressed_linear_forward(ctypes.byref(d), fake, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 1, fake, ws - 256,
+                                     None)
+    assert st == C.CQL_ERR_SIZE
+    st = L.compressed_linear_forward(ctypes.byref(d), fake, fake, C.CQL_DT_F32, fake, C.CQL_DT_F16, 1, fake, ws, None)
+    assert st == C.CQL_ERR_ARG                       # fp32 activations are not accepted
+    st = L.compressed_linear_forward(ctypes.byref(d), fake, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 0, fake, ws, None)
+    assert st == C.CQL_ERR_ARG
+    pw = C.cql_pack_workspace_size(d)
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, None, None, fake, lay.total_bytes, fake, pw,
+                                  None)
+    assert st == C.CQL_ERR_ARG                       # rank 16 needs L and R
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, fake, fake, fake, lay.total_bytes - 1, fake, pw,
+                                  None)
+    assert st == C.CQL_ERR_SIZE
+    st = L.pack_compressed_weight(ctypes.byref(d), fake + 8, C.CQL_DT_F32, fake, fake, fake, lay.total_bytes, fake, pw,
+                                  None)
+    assert st == C.CQL_ERR_ALIGN
+    assert L.cql_get_device_status(None, None, None) == C.CQL_ERR_ARG
+
+
+def test_workspace_sizes_grow_with_batch(lib):
+    d = C.make_desc(11008, 4096, rank=128)
+    sizes = [C.cql_workspace_size(d, b) for b in (1, 4, 16)]
+    assert sizes[0] < sizes[1] < sizes[2]
+    assert all(s % 256 == 0 for s in sizes)

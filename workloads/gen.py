@@ -32,10 +32,10 @@ import numpy as np
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round to nearest, ties to even); return the
     16-bit patterns.  NaN is not produced by the generators and not handled."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    u = u + np.uint64(0x7FFF) + lsb
-    return (u >> np.uint64(16)).astype(np.uint16)
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    u = u + np.uint32(0x7FFF) + lsb          # finite inputs: no 32-bit overflow
+    return (u >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
