@@ -1,0 +1,539 @@
+// Prefill path (batch > 16): Y = X deq(Q (.) M)^T + X R^T L^T on the 5th-gen
+// tensor cores (tcgen05.mma, kind::f16, bf16 operands, fp32 accumulators in
+// tensor memory), operands staged by TMA.
+//
+// Exactness.  A dequantised weight q*s has up to 14 significant bits; rounding
+// it to bf16 (8 bits) would cost ~1e-3 of relative error per output, most of
+// the 2e-3 budget.  So the GEMM never multiplies by q*s: the tensor cores see
+// the integer codes q (exact in bf16) and accumulate one scale group (128
+// columns of K) at a time in tensor memory; the epilogue warps multiply each
+// group's partial sums by that row's fp32 scale and add them into registers:
+//     Y^T[n][t] = sum_g s[n][g] * (sum_{k in g} q[n][k] X[t][k])
+// (SLiM-Quant's per-group scale, SLiM review summary "SLIM-Quant").  Weights
+// are the MMA's M side (one tensor-memory lane per output row), so the scale
+// is a per-thread scalar.  The low-rank term rides as three extra K blocks
+// with exact bf16 hi/lo splits, L^ T^T = Lhi Thi + Lhi Tlo + Llo Thi (SLiM
+// "Low-rank adapter quantization"; the adapters are AbsMax int4 g128).
+//
+// Kernels, in stream order:
+//   k_pf_dequant   packed planes -> q as bf16 (2:4 expanded, zeros where
+//                  pruned) [N][K + r3], fp32 scales [N][K/128], and the same
+//                  for R (rows padded to 128); L^ hi/lo in the extra columns.
+//   k_pf_gemm      T-pass: T = X R^T (split over K, fp32 atomics)
+//   k_pf_tsplit    T -> [Thi | Tlo | Thi] bf16, clears the accumulator
+//   k_pf_gemm      main pass: Y = ...
+// Roles inside k_pf_gemm (one CTA per SM, persistent over 128x256 tiles):
+//   warp 0        TMA producer (4-stage ring of A 128x64 and B 256x64 tiles)
+//   warp 1        tensor-memory allocator and single-thread MMA issuer
+//   warps 4..11   epilogue: tcgen05.ld, per-row group scale, stores
+// Every mbarrier wait is bounded; on expiry the kernel records
+// CQL_ERR_TIMEOUT in the error word and winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cql {
+
+constexpr int PF_BM = 128;        // weight rows per tile (MMA M, tensor-memory lanes)
+constexpr int PF_BN = 256;        // tokens per tile (MMA N)
+constexpr int PF_BK = 64;         // K per stage (one 128-byte swizzle row of bf16)
+constexpr int PF_STAGES = 4;
+constexpr int PF_THREADS = 384;
+constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;
+constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;
+constexpr uint32_t PF_WAIT_LIMIT = 1u << 26;
+
+struct PfGemmParams {
+  const float* scales;       // [rows][G] fp32
+  int rows;                  // weight rows (N, or R rows padded to 128)
+  int m;                     // tokens
+  int groups;                // K / 128
+  int lr_blocks;             // extra K blocks of 64 (main pass), 0 for the T pass
+  int k_splits;              // split of the group range (T pass)
+  int row_tiles, tok_tiles;
+  int mode;                  // 0: store y (out_dt), 1: atomic-add fp32 into out
+  void* out;
+  int out_dt;
+  int ldo;                   // leading dimension of out (elements)
+  int valid_rows;            // rows that produce output (N, or rank for the T pass)
+  uint32_t* err;
+};
+
+// ---------------------------------------------------------------------------
+// small PTX wrappers
+// ---------------------------------------------------------------------------
+CQL_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+CQL_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+CQL_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+CQL_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Bounded wait for the phase of the given parity; false if the limit ran out.
+CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t it = 0; it < PF_WAIT_LIMIT; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+CQL_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+CQL_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+CQL_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+CQL_DEV void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, 128 x 256 x 16, bf16 in, fp32 out.
+CQL_DEV void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+CQL_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+CQL_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile written by TMA with
+// 128-byte swizzling (8-row x 128-byte atoms, atoms 1024 bytes apart).
+CQL_DEV uint64_t smem_desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major,
+// M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PF_BN >> 3) << 17) |
+                            ((uint32_t)(PF_BM >> 4) << 24);
+
+// ---------------------------------------------------------------------------
+// the GEMM
+// ---------------------------------------------------------------------------
+struct PfSmem {
+  uint8_t a[PF_STAGES][PF_A_BYTES];
+  uint8_t b[PF_STAGES][PF_B_BYTES];
+  uint64_t full[PF_STAGES], empty[PF_STAGES];
+  uint64_t tfull[2], tempty[2];
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    k_pf_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmT, PfGemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PF_STAGES; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.tfull[b], 1);
+      mbar_init(&S.tempty[b], 8);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&S.tmem_base))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  const int n_items = p.row_tiles * p.tok_tiles * p.k_splits;
+  const int main_blocks = 2 * p.groups;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int split = item % p.k_splits, tile = item / p.k_splits;
+        const int rt = tile / p.tok_tiles, tt = tile % p.tok_tiles;
+        const int g0 = p.groups * split / p.k_splits, g1 = p.groups * (split + 1) / p.k_splits;
+        const int nkb = 2 * (g1 - g0) + (split == p.k_splits - 1 ? p.lr_blocks : 0);
+        for (int j = 0; j < nkb; ++j, ++it) {
+          const int s = it % PF_STAGES;
+          if (!mbar_wait(&S.empty[s], ((it / PF_STAGES) & 1) ^ 1)) { ok = false; break; }
+          mbar_expect_tx(&S.full[s], PF_A_BYTES + PF_B_BYTES);
+          const int kb = 2 * g0 + j;                       // absolute K block (LR blocks follow the main ones)
+          tma_load_2d(S.a[s], &tmA, &S.full[s], kb * PF_BK, rt * PF_BM);
+          if (kb < main_blocks) {
+            tma_load_2d(S.b[s], &tmB, &S.full[s], kb * PF_BK, tt * PF_BN);
+          } else {
+            tma_load_2d(S.b[s], &tmT, &S.full[s], (kb - main_blocks) * PF_BK, tt * PF_BN);
+          }
+        }
+      }
+      if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 10);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    if (lane == 0) {
+      uint32_t it = 0, gc = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int split = item % p.k_splits;
+        const int g0 = p.groups * split / p.k_splits, g1 = p.groups * (split + 1) / p.k_splits;
+        const int ngroups = (g1 - g0) + (split == p.k_splits - 1 && p.lr_blocks > 0 ? 1 : 0);
+        for (int g = 0; g < ngroups && ok; ++g, ++gc) {
+          const bool lr = g >= g1 - g0;
+          const int nkb = lr ? p.lr_blocks : 2;
+          const uint32_t buf = gc & 1;
+          if (!mbar_wait(&S.tempty[buf], ((gc >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + buf * PF_BN;
+          for (int j = 0; j < nkb; ++j, ++it) {
+            const int s = it % PF_STAGES;
+            if (!mbar_wait(&S.full[s], (it / PF_STAGES) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t da = smem_desc_sw128(smem_u32(S.a[s]));
+            const uint64_t db = smem_desc_sw128(smem_u32(S.b[s]));
+#pragma unroll
+            for (int kk = 0; kk < PF_BK / 16; ++kk)
+              tc_mma(d, da + 2 * kk, db + 2 * kk, kIdesc, (j > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&S.empty[s]);
+          }
+          tc_commit(&S.tfull[buf]);
+        }
+      }
+      if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 11);
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue ----------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    const int q = warp & 3, h = (warp - 4) >> 2;
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int split = item % p.k_splits, tile = item / p.k_splits;
+      const int rt = tile / p.tok_tiles, tt = tile % p.tok_tiles;
+      const int g0 = p.groups * split / p.k_splits, g1 = p.groups * (split + 1) / p.k_splits;
+      const int ngroups = (g1 - g0) + (split == p.k_splits - 1 && p.lr_blocks > 0 ? 1 : 0);
+      const int row = rt * PF_BM + 32 * q + lane;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      float s_next = (g0 < g1) ? __ldg(p.scales + (uint64_t)row * p.groups + g0) : 1.0f;
+      for (int g = 0; g < ngroups; ++g, ++gc) {
+        const float s = s_next;
+        const int gn = g0 + g + 1;
+        s_next = (g + 1 < g1 - g0) ? __ldg(p.scales + (uint64_t)row * p.groups + gn) : 1.0f;
+        const uint32_t buf = gc & 1;
+        if (!mbar_wait(&S.tfull[buf], (gc >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + buf * PF_BN + h * 128;
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+          float v0[32], v1[32];
+          tmem_ld32(base + c * 32, v0);
+          tmem_ld32(base + (c + 1) * 32, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            acc[c * 32 + i] = fmaf(s, v0[i], acc[c * 32 + i]);
+            acc[(c + 1) * 32 + i] = fmaf(s, v1[i], acc[(c + 1) * 32 + i]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.tempty[buf]);
+      }
+      if (!ok) break;
+      if (row < p.valid_rows) {
+        const int t0 = tt * PF_BN + h * 128;
+        if (p.mode == 0) {
+#pragma unroll 4
+          for (int i = 0; i < 128; ++i)
+            if (t0 + i < p.m) store_out(p.out, p.out_dt, (uint64_t)(t0 + i) * p.ldo + row, acc[i]);
+        } else {
+          float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll 4
+          for (int i = 0; i < 128; ++i)
+            if (t0 + i < p.m) atomicAdd(o + (uint64_t)(t0 + i) * p.ldo + row, acc[i]);
+        }
+      }
+    }
+    if (!ok && lane == 0) set_error(p.err, CQL_ERR_TIMEOUT, 12);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// dequantisation to exact bf16 codes (+ scales), adapters as hi/lo splits
+// ---------------------------------------------------------------------------
+CQL_DEV uint16_t bf16_bits_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+CQL_DEV uint16_t int_to_bf16(int q) { return bf16_bits_rn((float)q); }   // exact for |q| <= 256
+
+// One thread per (row, 128-column unit) of W: q codes -> bf16, zeros where the
+// 2:4 mask pruned; and the unit's scale as fp32.
+__global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* scales) {
+  const int G = p.upr;
+  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (uint64_t)p.d.n_out * G) return;
+  const int g = (int)(id / p.d.n_out), n = (int)(id % p.d.n_out);   // consecutive threads: consecutive rows
+  const int bits = codec_bits(p.d.codec);
+  const int bias = 1 << (bits - 1);
+  const uint32_t mask = (1u << bits) - 1;
+  uint16_t outv[128];
+  if (p.d.mask == CQL_MASK_2_4) {
+    // 64 kept codes (bits each) from bit 64*bits*g of the row stream, 32 pattern nibbles
+    const uint64_t bit0 = (uint64_t)64 * bits * g;
+    for (int gi = 0; gi < 32; ++gi) {
+      const uint32_t mb = p.meta[rit(n, (uint64_t)g * 16 + gi / 2, p.rb.meta)];
+      const uint32_t pt = (mb >> (4 * (gi & 1))) & 15u;
+      const int i0 = pt < 3 ? 0 : (pt < 5 ? 1 : 2);
+      const int i1 = pt == 0 ? 1 : (pt == 1 || pt == 3 ? 2 : 3);
+      int qv[2];
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t bp = bit0 + (uint64_t)bits * (2 * gi + h);
+        uint32_t c = 0;
+        for (int t = 0; t < bits; ++t) {
+          const uint64_t sb = bp + t;
+          c |= ((uint32_t)(p.values[rit(n, sb >> 3, p.rb.values)] >> (sb & 7)) & 1u) << t;
+        }
+        qv[h] = (int)(c & mask) - bias;
+      }
+      for (int i = 0; i < 4; ++i) outv[4 * gi + i] = 0;
+      outv[4 * gi + i0] = int_to_bf16(qv[0]);
+      outv[4 * gi + i1] = int_to_bf16(qv[1]);
+    }
+  } else {
+    const uint64_t bit0 = (uint64_t)128 * bits * g;
+    for (int c = 0; c < 128; ++c) {
+      const uint64_t bp = bit0 + (uint64_t)bits * c;
+      uint32_t code = 0;
+      for (int t = 0; t < bits; ++t) {
+        const uint64_t sb = bp + t;
+        code |= ((uint32_t)(p.values[rit(n, sb >> 3, p.rb.values)] >> (sb & 7)) & 1u) << t;
+      }
+      outv[c] = int_to_bf16((int)code - bias);
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + (uint64_t)g * 128);
+  for (int i = 0; i < 16; ++i) {
+    uint4 v;
+    v.x = outv[8 * i + 0] | ((uint32_t)outv[8 * i + 1] << 16);
+    v.y = outv[8 * i + 2] | ((uint32_t)outv[8 * i + 3] << 16);
+    v.z = outv[8 * i + 4] | ((uint32_t)outv[8 * i + 5] << 16);
+    v.w = outv[8 * i + 6] | ((uint32_t)outv[8 * i + 7] << 16);
+    dst[i] = v;
+  }
+  scales[(uint64_t)n * G + g] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(p.scales + rit(n, 2 * g, p.rb.scales)));
+}
+
+// Adapter columns of the main operand: [Lhi | Lhi | Llo | 0] at columns
+// K .. K + r3 of row n, with L^ = q_L s_L exact in fp32 and Lhi + Llo = L^.
+__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3) {
+  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int r = p.d.rank;
+  if (id >= (uint64_t)p.d.n_out * r3) return;
+  const int n = (int)(id / r3), c = (int)(id % r3);
+  uint16_t v = 0;
+  if (c < 3 * r) {
+    const int j = c % r, part = c / r;                       // 0: hi, 1: hi, 2: lo
+    const uint32_t byte = p.l_values[rit(n, j / 2, p.rb.l_values)];
+    const int q = (int)((byte >> (4 * (j & 1))) & 15u) - 8;
+    const float s = f16_bits_to_f32(p.l_scales[(uint64_t)(n / kGroup) * r + j]);
+    const float l = (float)q * s;                            // exact (<= 14 significant bits)
+    const uint16_t hi = bf16_bits_rn(l);
+    v = part < 2 ? hi : bf16_bits_rn(l - bf16_bits_to_f32(hi));
+  }
+  qbf[(uint64_t)n * ldq + p.d.k_in + c] = v;
+}
+
+// R rows (padded to 128) as bf16 codes and fp32 scales.
+__global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, int rows) {
+  const int K = p.d.k_in, G = p.upr;
+  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (uint64_t)rows * K) return;
+  const int j = (int)(id / K), k = (int)(id % K);
+  uint16_t v = 0;
+  if (j < p.d.rank) {
+    const uint32_t byte = p.r_values[rit(j, k / 2, p.rb.r_values)];
+    v = int_to_bf16((int)((byte >> (4 * (k & 1))) & 15u) - 8);
+  }
+  rbf[id] = v;
+  if (k % kGroup == 0)
+    rscales[(uint64_t)j * G + k / kGroup] =
+        j < p.d.rank ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(p.r_scales + rit(j, 2 * (k / kGroup), p.rb.r_scales)))
+                     : 0.0f;
+}
+
+// T [m][r_pad] fp32 -> [Thi | Tlo | Thi | 0] bf16 [m][r3]; clears T.
+__global__ void k_pf_tsplit(float* t, int ldt, uint16_t* t3, int r3, int r, int m) {
+  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (uint64_t)m * r3) return;
+  const int row = (int)(id / r3), c = (int)(id % r3);
+  uint16_t v = 0;
+  if (c < 3 * r) {
+    const int j = c % r, part = c / r;                       // 0: hi, 1: lo, 2: hi
+    const float x = t[(uint64_t)row * ldt + j];
+    const uint16_t hi = bf16_bits_rn(x);
+    v = part == 1 ? bf16_bits_rn(x - bf16_bits_to_f32(hi)) : hi;
+  }
+  t3[id] = v;
+  __syncthreads();
+  if (c < r && c < ldt) t[(uint64_t)row * ldt + c] = 0.0f;   // thread (row, c) read (row, c % r) only for c < 3r
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major, ld elements) with a box of
+// box_rows x 64 columns, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {PF_BK, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+PrefillLayout prefill_layout(const cql_desc& d, int m) {
+  PrefillLayout L{};
+  const uint64_t n = (uint64_t)d.n_out, k = (uint64_t)d.k_in, r = (uint64_t)d.rank;
+  L.r3 = r ? (int)((3 * r + 63) / 64 * 64) : 0;
+  L.rrows = r ? (int)((r + 127) / 128 * 128) : 0;
+  L.r_pad = (int)((r + 31) / 32 * 32);
+  L.ldq = (int)(k + L.r3);
+  uint64_t pos = 0;
+  L.qbf = pos;     pos = align256(pos + n * L.ldq * 2);
+  L.wsc = pos;     pos = align256(pos + n * (k / 128) * 4);
+  L.rbf = pos;     pos = align256(pos + (uint64_t)L.rrows * k * 2);
+  L.rsc = pos;     pos = align256(pos + (uint64_t)L.rrows * (k / 128) * 4);
+  L.tacc = pos;    pos = align256(pos + (uint64_t)m * L.r_pad * 4);
+  L.t3 = pos;      pos = align256(pos + (uint64_t)m * L.r3 * 2);
+  L.total = pos;
+  return L;
+}
+
+static int sm_count_pf() {
+  int dev = 0, v = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  return v > 0 ? v : 148;
+}
+
+cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st) {
+  const PrefillLayout L = prefill_layout(p.d, p.batch);
+  const int N = p.d.n_out, K = p.d.k_in, r = p.d.rank, m = p.batch, G = p.upr;
+  uint16_t* qbf = reinterpret_cast<uint16_t*>(pws + L.qbf);
+  float* wsc = reinterpret_cast<float*>(pws + L.wsc);
+  uint16_t* rbf = reinterpret_cast<uint16_t*>(pws + L.rbf);
+  float* rsc = reinterpret_cast<float*>(pws + L.rsc);
+  float* tacc = reinterpret_cast<float*>(pws + L.tacc);
+  uint16_t* t3 = reinterpret_cast<uint16_t*>(pws + L.t3);
+  const bool lowrank = r > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
+  const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
+
+  static bool attr_set = false;
+  const size_t smem = sizeof(PfSmem) + 1024;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute((const void*)k_pf_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const uint64_t nw = (uint64_t)N * G;
+  k_pf_dequant_w<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc);
+  if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);       // main term off: zero scales
+  if (lowrank) {
+    const uint64_t nl = (uint64_t)N * L.r3;
+    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.r3);
+    const uint64_t nr = (uint64_t)L.rrows * K;
+    k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count_pf();
+  CUtensorMap mA, mB, mT, mR;
+  if (!make_map(&mB, p.x, (uint64_t)m, (uint64_t)K, (uint64_t)K, PF_BN)) return cudaErrorInvalidValue;
+  if (lowrank) {
+    // T pass: T = X R^T, split over K, fp32 atomics into tacc (zero on entry)
+    if (!make_map(&mR, rbf, (uint64_t)L.rrows, (uint64_t)K, (uint64_t)K, PF_BM)) return cudaErrorInvalidValue;
+    PfGemmParams t{};
+    t.scales = rsc; t.rows = L.rrows; t.m = m; t.groups = G; t.lr_blocks = 0;
+    t.row_tiles = L.rrows / PF_BM; t.tok_tiles = (m + PF_BN - 1) / PF_BN;
+    const int tiles = t.row_tiles * t.tok_tiles;
+    t.k_splits = max(1, min(G, sms / max(tiles, 1)));
+    t.mode = 1; t.out = tacc; t.out_dt = CQL_DT_F32; t.ldo = L.r_pad; t.valid_rows = r; t.err = p.err;
+    const int items = tiles * t.k_splits;
+    k_pf_gemm<<<min(items, sms), PF_THREADS, smem, st>>>(mR, mB, mB, t);
+    const uint64_t nt = (uint64_t)m * L.r3;
+    k_pf_tsplit<<<(unsigned)((nt + 255) / 256), 256, 0, st>>>(tacc, L.r_pad, t3, L.r3, r, m);
+    if (!make_map(&mT, t3, (uint64_t)m, (uint64_t)L.r3, (uint64_t)L.r3, PF_BN)) return cudaErrorInvalidValue;
+  } else {
+    mT = mB;
+  }
+  if (!make_map(&mA, qbf, (uint64_t)N, (uint64_t)L.ldq, (uint64_t)L.ldq, PF_BM)) return cudaErrorInvalidValue;
+  PfGemmParams g{};
+  g.scales = wsc; g.rows = N; g.m = m; g.groups = G; g.lr_blocks = lowrank ? L.r3 / PF_BK : 0;
+  g.row_tiles = N / PF_BM; g.tok_tiles = (m + PF_BN - 1) / PF_BN; g.k_splits = 1;
+  g.mode = 0; g.out = p.y; g.out_dt = p.ydt; g.ldo = N; g.valid_rows = N; g.err = p.err;
+  const int items = g.row_tiles * g.tok_tiles;
+  k_pf_gemm<<<min(items, sms), PF_THREADS, smem, st>>>(mA, mB, mT, g);
+  return cudaGetLastError();
+}
+
+}  // namespace cql
