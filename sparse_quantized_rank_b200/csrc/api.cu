@@ -123,6 +123,7 @@ ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch) {
   w.t_part = pos;    pos = align256(pos + upr * bp * rpad * 4);
   w.t_final = pos;   pos = align256(pos + bp * rpad * 4);
   w.prefill = pos;
+  if (batch > CQL_MAX_DECODE_BATCH) pos = align256(pos + prefill_layout(d, batch).total);
   w.total = pos;
   return w;
 }
@@ -245,7 +246,7 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   if (!aligned(packed, 256) || !aligned(workspace, 256) || !aligned(x, 16) || !aligned(y, 16)) return CQL_ERR_ALIGN;
   const ForwardWorkspace fw = forward_workspace_layout(d, batch);
   if (ws_bytes < fw.total) return CQL_ERR_SIZE;
-  if (batch > CQL_MAX_DECODE_BATCH) return CQL_ERR_UNSUPPORTED;
+  if (batch > CQL_MAX_DECODE_BATCH && !prefill_supported(d, x_dt)) return CQL_ERR_UNSUPPORTED;
 
   cql_layout lay;
   compute_layout(d, &lay);
@@ -284,7 +285,9 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   p.counters = reinterpret_cast<uint32_t*>(ws + fw.counters);
   p.t_part = reinterpret_cast<float*>(ws + fw.t_part);
   p.t_final = reinterpret_cast<float*>(ws + fw.t_final);
-  const cudaError_t e = launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e = batch > CQL_MAX_DECODE_BATCH
+                            ? launch_prefill(p, ws + fw.prefill, reinterpret_cast<cudaStream_t>(stream))
+                            : launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CQL_OK : CQL_ERR_CUDA;
 }
 

@@ -31,28 +31,57 @@
 
 namespace cql {
 
-constexpr int kDecNT = 512;                    // threads per decode CTA
-// Batch 1 runs two CTAs per SM (64 registers per thread, <= 100 KB of tables
-// each); larger batches need more accumulator registers and run one CTA per
-// SM with up to 200 KB of tables.
+constexpr int kDecNT = 512;                    // threads per decode CTA (one CTA per SM)
+constexpr int kDecNW = kDecNT / 32;
+constexpr int kDepth = 4;                      // units in flight per warp (cp.async ring)
+constexpr int kDecSmem = 220 * 1024;           // shared memory per CTA: tables + ring
 template <int B> struct DecCfg {
-  static constexpr int kMinBlocks = B == 1 ? 2 : 1;
-  static constexpr int kSmemBudget = B == 1 ? 100 * 1024 : 200 * 1024;
+  static constexpr int kMinBlocks = 1;
 };
 constexpr uint32_t kMagic = 0x4B000000u;       // fp32 bit pattern of 2^23
 
 CQL_DEV float act(const DecodeParams& p, int b, int col) {
   return b < p.batch ? to_f32_act(p.x, p.xdt, (uint64_t)b * p.d.k_in + col) : 0.0f;
 }
-CQL_DEV uint32_t ldg_u16(const uint8_t* p) { return __ldg(reinterpret_cast<const unsigned short*>(p)); }
+
+CQL_DEV void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+CQL_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+CQL_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+CQL_DEV uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// Activations x[b][c0, c0 + ncols) -> fp32 xs[c * B + b] in shared memory,
+// eight columns per 16-byte load (ncols is a multiple of 128; rows of x are
+// 16-byte aligned).  Batch rows beyond p.batch are zero.
+template <int B>
+CQL_DEV void stage_x(const DecodeParams& p, float* xs, int c0, int ncols) {
+  const int chunks = ncols >> 3;
+  const uint16_t* xb = static_cast<const uint16_t*>(p.x);
+  for (int i = threadIdx.x; i < B * chunks; i += blockDim.x) {
+    const int b = i / chunks, ch = i - b * chunks;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (b < p.batch) w = *reinterpret_cast<const uint4*>(xb + (uint64_t)b * p.d.k_in + c0 + 8 * ch);
+    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t h = (wd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+      xs[(8 * ch + j) * B + b] = p.xdt == CQL_DT_BF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
+    }
+  }
+}
 
 // ---------------------------------------------------------------------------
 // epilogue for one row block: accumulator + CSR + low rank -> y
 // ---------------------------------------------------------------------------
 template <int B>
 CQL_DEV void finish_rowblock(const DecodeParams& p, int rb, int lane) {
-  const int N = p.d.n_out, K = p.d.k_in;
+  const int N = p.d.n_out;
   const int row = rb * 32 + lane;
+  if (p.has_pre) pdl_wait();            // CSR rows and t = R_q x are complete
   float acc[B];
 #pragma unroll
   for (int b = 0; b < B; ++b) {
@@ -63,22 +92,11 @@ CQL_DEV void finish_rowblock(const DecodeParams& p, int rb, int lane) {
       *a = 0.0f;
     }
   }
-  if (p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR)) {
-    int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
-    e0 = max(0, min(e0, (int)p.nnz));
-    e1 = max(e0, min(e1, (int)p.nnz));
-    for (int e = e0; e < e1; ++e) {
-      const int col = p.csr_col[e];
-      if (col >= K) continue;
-      const float v = f16_bits_to_f32(p.csr_val[e]);
-#pragma unroll
-      for (int b = 0; b < B; ++b) acc[b] = fmaf(v, act(p, b, col), acc[b]);
-    }
-  }
   if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK)) {
-    pdl_wait();                                   // stage 1 (t = R_q x) complete
     const int r = p.d.rank, g = row / kGroup;
-    for (int m = 0; m * 32 < r; ++m) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {             // rank <= 256: at most 8 chunks of 32
+      if (32 * m >= r) break;
       const int j = 32 * m + lane;
       float u[B];
       const float ls = j < r ? f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) : 0.0f;
@@ -133,49 +151,64 @@ template <int BITS, int B>
 struct Unit24 {
   static constexpr int NBP = B == 1 ? 1 : B / 2;                     // batch pairs
   static constexpr int kGroupBytes = B == 1 ? 64 : 128 * NBP;        // 8 patterns per group
-  static constexpr int kUnitBytes = 32 * kGroupBytes;
+  static constexpr int kTableBytes = 32 * kGroupBytes;
+  static constexpr int kUnitBytes = kTableBytes + kGroup * B * 4;   // table + staged x
   struct Frag {
     uint32_t v[8];
     uint32_t m[4];
     uint32_t s;
   };
 
+  // Pair table of the K tile: entry (group, pattern) = the x values of the
+  // pattern's two kept columns (B == 1), or of two batches (B >= 2).
   static CQL_DEV void build(const DecodeParams& p, uint8_t* smem, int kt) {
     const int c0 = kt * p.ktu * kGroup;
-    const int ngroups = min(p.ktu, p.upr - kt * p.ktu) * (kGroup / 4);
+    const int units = min(p.ktu, p.upr - kt * p.ktu);
+    const int ngroups = units * (kGroup / 4);
+    float* xs = reinterpret_cast<float*>(smem + (size_t)p.ktu * kTableBytes);
+    stage_x<B>(p, xs, c0, units * kGroup);
+    __syncthreads();
     for (int i = threadIdx.x; i < ngroups * NBP * 6; i += blockDim.x) {
       const int pt = i % 6, t2 = i / 6, bp = t2 % NBP, g = t2 / NBP;
       int i0, i1;
       pair_of(pt, i0, i1);
-      const int col = c0 + 4 * g;
+      const float* xc = xs + (4 * g) * B;
       if (B == 1) {
-        *reinterpret_cast<float2*>(smem + g * 64 + pt * 8) = make_float2(act(p, 0, col + i0), act(p, 0, col + i1));
+        *reinterpret_cast<float2*>(smem + g * 64 + pt * 8) = make_float2(xc[i0], xc[i1]);
       } else {
         const int b = 2 * bp;
         *reinterpret_cast<float4*>(smem + ((g * NBP + bp) * 8 + pt) * 16) =
-            make_float4(act(p, b, col + i0), act(p, b, col + i1), act(p, b + 1, col + i0), act(p, b + 1, col + i1));
+            make_float4(xc[i0 * B + b], xc[i1 * B + b], xc[i0 * B + b + 1], xc[i1 * B + b + 1]);
       }
     }
   }
   static CQL_DEV void on_row(const DecodeParams&, uint8_t*, int, int) {}
 
-  static CQL_DEV void load(const DecodeParams& p, int rb, int uk, int lane, Frag& f) {
+  // Stage one unit: its code slabs and pattern slab (cp.async into this
+  // lane's 16-byte column of the slot); returns the scale (and, for 3-bit
+  // codes, whether the unit starts mid-slab).
+  static constexpr int kSlabs = 3;
+  static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
+    const uint32_t vs = BITS == 4 ? 2u * uk : (24u * uk) >> 4;
+    const uint8_t* vb = p.values + slab_off(rb, vs, p.rb.values) + lane * 16;
+    cp_async16(slot, vb);
+    cp_async16(slot + 512, vb + 512);
+    cp_async16(slot + 1024, p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
+    const uint32_t sc = ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    return sc | (BITS == 3 && ((24u * uk) & 15u) ? 0x10000u : 0u);
+  }
+  static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
+    const uint4 a = lds128(slot), b = lds128(slot + 512), m = lds128(slot + 1024);
     if (BITS == 4) {
-      const uint8_t* vb = p.values + slab_off(rb, 2 * uk, p.rb.values) + lane * 16;
-      const uint4 a = ldg_stream(vb), b = ldg_stream(vb + 512);
       f.v[0] = a.x; f.v[1] = a.y; f.v[2] = a.z; f.v[3] = a.w;
       f.v[4] = b.x; f.v[5] = b.y; f.v[6] = b.z; f.v[7] = b.w;
     } else {
-      const uint32_t byte0 = 24u * uk;
-      const uint8_t* vb = p.values + slab_off(rb, byte0 >> 4, p.rb.values) + lane * 16;
-      const uint4 a = ldg_stream(vb), b = ldg_stream(vb + 512);
-      const bool odd = (byte0 & 15u) != 0;          // codes start at bit 64 of the window
+      const bool odd = (sc >> 16) & 1u;             // codes start at bit 64 of the window
       f.v[0] = odd ? a.z : a.x; f.v[1] = odd ? a.w : a.y; f.v[2] = odd ? b.x : a.z; f.v[3] = odd ? b.y : a.w;
       f.v[4] = odd ? b.z : b.x; f.v[5] = odd ? b.w : b.y; f.v[6] = b.z; f.v[7] = b.w;
     }
-    const uint4 m = ldg_stream(p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
     f.m[0] = m.x; f.m[1] = m.y; f.m[2] = m.z; f.m[3] = m.w;
-    f.s = ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    f.s = sc & 0xFFFFu;
   }
 
   template <int J>
@@ -226,7 +259,7 @@ struct Unit24 {
 
   static CQL_DEV void compute(const DecodeParams& p, const uint8_t* smem, const Frag& f, int ut, int lane,
                               float (&acc)[B]) {
-    const uint8_t* tb = smem + (size_t)ut * kUnitBytes;
+    const uint8_t* tb = smem + (size_t)ut * kTableBytes;
     uint64_t a2[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) a2[b] = 0;
@@ -256,8 +289,7 @@ struct UnitDense {
   static CQL_DEV void build(const DecodeParams& p, uint8_t* smem, int kt) {
     const int c0 = kt * p.ktu * kGroup;
     const int ncols = min(p.ktu, p.upr - kt * p.ktu) * kGroup;
-    float* xs = reinterpret_cast<float*>(smem);
-    for (int i = threadIdx.x; i < ncols * B; i += blockDim.x) xs[i] = act(p, i % B, c0 + i / B);
+    stage_x<B>(p, reinterpret_cast<float*>(smem), c0, ncols);
   }
   static CQL_DEV void on_row(const DecodeParams& p, uint8_t* smem, int rb, int lane) {
     if (!LUT) return;
@@ -267,15 +299,20 @@ struct UnitDense {
     for (int c = 0; c < (1 << BITS); ++c) lut[c * 32 + lane] = f16_bits_to_f32(ldg_u16(p.scales + rit(row, 2 * c, p.rb.scales)));
     __syncwarp();
   }
-  static CQL_DEV void load(const DecodeParams& p, int rb, int uk, int lane, Frag& f) {
-    constexpr int slabs = BITS;                            // 64 or 48 bytes per unit
-    const uint8_t* vb = p.values + slab_off(rb, (uint64_t)slabs * uk, p.rb.values) + lane * 16;
+  static constexpr int kSlabs = BITS;                     // 64 or 48 bytes of codes per unit
+  static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
+    const uint8_t* vb = p.values + slab_off(rb, (uint64_t)BITS * uk, p.rb.values) + lane * 16;
 #pragma unroll
-    for (int s = 0; s < slabs; ++s) {
-      const uint4 a = ldg_stream(vb + 512 * s);
+    for (int s = 0; s < BITS; ++s) cp_async16(slot + 512 * s, vb + 512 * s);
+    return LUT ? 0u : ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+  }
+  static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
+#pragma unroll
+    for (int s = 0; s < BITS; ++s) {
+      const uint4 a = lds128(slot + 512 * s);
       f.v[4 * s + 0] = a.x; f.v[4 * s + 1] = a.y; f.v[4 * s + 2] = a.z; f.v[4 * s + 3] = a.w;
     }
-    f.s = LUT ? 0u : ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    f.s = sc;
   }
   template <int C>
   static CQL_DEV uint32_t code(const Frag& f) {
@@ -338,16 +375,20 @@ struct UnitBitmap {
   static CQL_DEV void build(const DecodeParams& p, uint8_t* smem, int kt) {
     const int c0 = kt * p.ktu * kGroup;
     const int ncols = min(p.ktu, p.upr - kt * p.ktu) * kGroup;
-    float* xs = reinterpret_cast<float*>(smem);
-    for (int i = threadIdx.x; i < ncols * B; i += blockDim.x) xs[i] = act(p, i % B, c0 + i / B);
+    stage_x<B>(p, reinterpret_cast<float*>(smem), c0, ncols);
   }
   static CQL_DEV void on_row(const DecodeParams&, uint8_t*, int, int) {}
-  static CQL_DEV void load(const DecodeParams& p, int rb, int uk, int lane, Frag& f) {
-    const uint4 m = ldg_stream(p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
-    f.bm[0] = m.x; f.bm[1] = m.y; f.bm[2] = m.z; f.bm[3] = m.w;
+  static constexpr int kSlabs = 1;                        // the unit's bitmap slab
+  static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
+    cp_async16(slot, p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
     const uint64_t row = (uint64_t)rb * 32 + lane;
-    f.voff = ldg_u16(p.voff + rit(row, 2 * uk, p.rb.voff));
-    f.s = ldg_u16(p.scales + rit(row, 2 * uk, p.rb.scales));
+    return ldg_u16(p.voff + rit(row, 2 * uk, p.rb.voff)) | (ldg_u16(p.scales + rit(row, 2 * uk, p.rb.scales)) << 16);
+  }
+  static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
+    const uint4 m = lds128(slot);
+    f.bm[0] = m.x; f.bm[1] = m.y; f.bm[2] = m.z; f.bm[3] = m.w;
+    f.voff = sc & 0xFFFFu;
+    f.s = sc >> 16;
   }
   static CQL_DEV void compute(const DecodeParams& p, uint8_t* smem, const Frag& f, int ut, int lane, int rb,
                               float (&acc)[B]) {
@@ -431,11 +472,12 @@ CQL_DEV bool header_ok(const DecodeParams& p) {
 }
 
 template <class U, int B>
-__global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(DecodeParams p) {
+__global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(DecodeParams p, int ring_off) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int NW = kDecNT / 32;
   if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
+  // this warp's ring of kDepth unit slots; lane l owns bytes [16 l, 16 l + 16) of every 512-byte slab
+  uint8_t* ring = smem + ring_off + (size_t)warp * (kDepth * U::kSlabs * 512) + lane * 16;
   const uint64_t U_ = p.n_units;
   const uint64_t ubeg = U_ * blockIdx.x / gridDim.x, uend = U_ * (blockIdx.x + 1) / gridDim.x;
   uint64_t u = ubeg;
@@ -448,26 +490,50 @@ __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(Decode
     U::build(p, smem, kt);
     __syncthreads();
     const uint64_t n = tend - u;
-    const uint64_t wb = u + n * warp / NW, we = u + n * (warp + 1) / NW;
+    const uint64_t wb = u + n * warp / kDecNW, we = u + n * (warp + 1) / kDecNW;
     if (wb < we) {
       int kt0, cur_rb, cur_ut;
       unit_coords(p, wb, kt0, cur_rb, cur_ut);
       const int ts = tile_size(p, kt);
       const int uk0 = kt * p.ktu;
-      typename U::Frag cur, nxt;
-      U::load(p, cur_rb, uk0 + cur_ut, lane, cur);
+      // prologue: stage the first kDepth units
+      int irb = cur_rb, iut = cur_ut;
+      uint32_t sc[kDepth];
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        sc[d] = 0;
+        if (wb + d < we) {
+          sc[d] = U::issue(p, irb, uk0 + iut, lane, ring + d * (U::kSlabs * 512));
+          if (++iut == ts) { iut = 0; ++irb; }
+        }
+        cp_async_commit();
+      }
       U::on_row(p, smem, cur_rb, lane);
       float acc[B];
 #pragma unroll
       for (int b = 0; b < B; ++b) acc[b] = 0.0f;
       uint32_t cnt = 0;
+      int slot = 0;
       for (uint64_t i = wb; i < we; ++i) {
+        uint8_t* sl = ring + slot * (U::kSlabs * 512);
+        cp_async_wait<kDepth - 1>();
+        __syncwarp();
+        typename U::Frag f;
+        U::gather(sl, sc[0], f);
+        __syncwarp();                               // slot contents are in registers
+#pragma unroll
+        for (int d = 0; d + 1 < kDepth; ++d) sc[d] = sc[d + 1];
+        if (i + kDepth < we) {
+          sc[kDepth - 1] = U::issue(p, irb, uk0 + iut, lane, sl);
+          if (++iut == ts) { iut = 0; ++irb; }
+        }
+        cp_async_commit();
+        if (++slot == kDepth) slot = 0;
+        Call<U, B>::compute(p, smem, f, cur_ut, lane, cur_rb, acc);
+        ++cnt;
         int nrb = cur_rb, nut = cur_ut + 1;
         if (nut == ts) { nut = 0; ++nrb; }
         const bool more = i + 1 < we;
-        if (more) U::load(p, nrb, uk0 + nut, lane, nxt);
-        Call<U, B>::compute(p, smem, cur, cur_ut, lane, cur_rb, acc);
-        ++cnt;
         if (!more || nrb != cur_rb) {
           flush_rowblock<B>(p, cur_rb, cnt, acc, lane);
 #pragma unroll
@@ -475,11 +541,11 @@ __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(Decode
           cnt = 0;
           if (more) U::on_row(p, smem, nrb, lane);
         }
-        cur = nxt;
         cur_rb = nrb;
         cur_ut = nut;
       }
     }
+    cp_async_wait<0>();
     u = tend;
   }
 }
@@ -495,51 +561,112 @@ __global__ void __launch_bounds__(256, 1) k_finish_only(DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// low-rank stage 1: t = deq(R_q) x  (one CTA per 128-column group, a warp per
-// 32 adapter rows), deterministic final sum by the last CTA
+// pre-kernel, PDL primary of the decode kernel:
+//  * blocks [0, n_s1): low-rank stage 1, t = deq(R_q) x.  Block (R row block,
+//    K slice of up to 8 units): a warp per unit, partial sums reduced in shared
+//    memory, per-slice partials; the last block to finish sums the slices in
+//    a fixed order into t_final (deterministic).
+//  * blocks [n_s1, ..): the CSR outliers, a thread per output row, added into
+//    the fp32 accumulator (SqueezeLLM "Approach": the sparse part of the
+//    dense-and-sparse decomposition).
+// The decode kernel's epilogue waits for this grid (griddepcontrol.wait)
+// before it reads the accumulator or t_final.
 // ---------------------------------------------------------------------------
+constexpr int kS1Units = 8;
+
 template <int B>
-__global__ void __launch_bounds__(256, 1) k_lowrank_stage1(DecodeParams p) {
+__global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
   pdl_launch_dependents();
-  __shared__ float xs[B][kGroup];
+  extern __shared__ __align__(16) float s1[];
   __shared__ bool s_last;
-  const int g = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < B * kGroup; i += blockDim.x) xs[i / kGroup][i % kGroup] = act(p, i / kGroup, g * kGroup + i % kGroup);
-  __syncthreads();
-  for (int w = warp; w < p.r_pad / 32; w += blockDim.x / 32) {
-    const uint8_t* base = p.r_values + slab_off(w, 4 * g, p.rb.r_values) + lane * 16;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x < n_s1) {
+    const int KQ = (p.upr + kS1Units - 1) / kS1Units;
+    const int rbR = blockIdx.x / KQ, kq = blockIdx.x % KQ;
+    const int u0 = kq * kS1Units, u1 = min(p.upr, u0 + kS1Units);
+    stage_x<B>(p, s1, u0 * kGroup, (u1 - u0) * kGroup);
+    __syncthreads();
     float acc[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+    const int j = 32 * rbR + lane;
+    for (int u = u0 + warp; u < u1; u += 8) {
+      const uint8_t* base = p.r_values + slab_off(rbR, 4 * u, p.rb.r_values) + lane * 16;
+      uint4 q4[4];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const uint4 q4 = ldg_stream(base + 512 * s);
-      const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
+      for (int s = 0; s < 4; ++s) q4[s] = ldg_stream(base + 512 * s);
+      const float sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit(j, 2 * u, p.rb.r_scales)));
+      const float* xs = s1 + (u - u0) * kGroup * B;
+      float au[B];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float q = (float)((int)((wd[k >> 3] >> (4 * (k & 7))) & 15u) - 8);
+      for (int b = 0; b < B; ++b) au[b] = 0.0f;
 #pragma unroll
-        for (int b = 0; b < B; ++b) acc[b] = fmaf(q, xs[b][32 * s + k], acc[b]);
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t wd[4] = {q4[s].x, q4[s].y, q4[s].z, q4[s].w};
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float q = (float)((int)((wd[k >> 3] >> (4 * (k & 7))) & 15u) - 8);
+#pragma unroll
+          for (int b = 0; b < B; ++b) au[b] = fmaf(q, xs[(32 * s + k) * B + b], au[b]);
+        }
       }
-    }
-    const int j = 32 * w + lane;
-    const float sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit(j, 2 * g, p.rb.r_scales)));
 #pragma unroll
-    for (int b = 0; b < B; ++b) p.t_part[((uint64_t)g * B + b) * p.r_pad + j] = acc[b] * sc;
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(p.t_counter, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    for (int i = threadIdx.x; i < B * p.r_pad; i += blockDim.x) {
-      const int b = i / p.r_pad, j = i % p.r_pad;
-      float s = 0.0f;
-      for (int gg = 0; gg < (int)gridDim.x; ++gg) s += ld_cg_f32(p.t_part + ((uint64_t)gg * B + b) * p.r_pad + j);
-      p.t_final[(uint64_t)b * p.r_pad + j] = s;
+      for (int b = 0; b < B; ++b) acc[b] = fmaf(sc, au[b], acc[b]);
     }
-    if (threadIdx.x == 0) *p.t_counter = 0u;
+    __syncthreads();                                   // x no longer needed: reuse for partials
+#pragma unroll
+    for (int b = 0; b < B; ++b) s1[(warp * B + b) * 32 + lane] = acc[b];
+    __syncthreads();
+    for (int i = threadIdx.x; i < B * 32; i += blockDim.x) {
+      const int b = i >> 5, l = i & 31;
+      float t = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) t += s1[(w * B + b) * 32 + l];
+      p.t_part[((uint64_t)kq * B + b) * p.r_pad + 32 * rbR + l] = t;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(p.t_counter, 1u) == (uint32_t)n_s1 - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int i = threadIdx.x; i < B * p.r_pad; i += blockDim.x) {
+        const int b = i / p.r_pad, jj = i - b * p.r_pad;
+        float t = 0.0f;
+#pragma unroll 4
+        for (int k2 = 0; k2 < KQ; ++k2) t += ld_cg_f32(p.t_part + ((uint64_t)k2 * B + b) * p.r_pad + jj);
+        p.t_final[(uint64_t)b * p.r_pad + jj] = t;
+      }
+      if (threadIdx.x == 0) *p.t_counter = 0u;
+    }
+  } else {
+    const int row = (blockIdx.x - n_s1) * blockDim.x + threadIdx.x;
+    if (row >= p.d.n_out) return;
+    int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
+    e0 = max(0, min(e0, (int)p.nnz));
+    e1 = max(e0, min(e1, (int)p.nnz));
+    if (e1 == e0) return;
+    float acc[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+    for (int e = e0; e < e1; e += 8) {
+      int col[8];
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool ok = e + i < e1;
+        col[i] = ok ? (int)p.csr_col[e + i] : 0;
+        v[i] = ok ? f16_bits_to_f32(p.csr_val[e + i]) : 0.0f;
+        if (col[i] >= p.d.k_in) { col[i] = 0; v[i] = 0.0f; }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[b] = fmaf(v[i], act(p, b, col[i]), acc[b]);
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+      if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
   }
 }
 
@@ -561,11 +688,13 @@ static int sm_count() {
 
 template <class U, int B>
 static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, cudaStream_t st, bool pdl) {
-  int ktu = (DecCfg<B>::kSmemBudget - extra_bytes) / unit_bytes;
+  const int ring = kDecNW * kDepth * U::kSlabs * 512;
+  int ktu = (kDecSmem - ring - extra_bytes) / unit_bytes;
   ktu = max(1, min(ktu, p.upr));
   p.ktu = ktu;
   p.n_tiles = (p.upr + ktu - 1) / ktu;
-  const size_t smem = (size_t)ktu * unit_bytes + extra_bytes;
+  const int ring_off = ktu * unit_bytes + extra_bytes;
+  const size_t smem = (size_t)ring_off + ring;
   static bool attr_set = false;       // once per instantiation: allow the opt-in maximum
   if (!attr_set) {
     int dev = 0, optin = 0;
@@ -576,8 +705,7 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int per_sm = DecCfg<B>::kMinBlocks;
-  uint64_t grid = (uint64_t)sm_count() * per_sm;
+  uint64_t grid = (uint64_t)sm_count() * DecCfg<B>::kMinBlocks;
   if (grid > p.n_units) grid = p.n_units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -589,14 +717,28 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_decode<U, B>, p);
+  return cudaLaunchKernelEx(&cfg, k_decode<U, B>, p, ring_off);
 }
 
 template <int B>
-static cudaError_t launch_decode_b(const DecodeParams& p, cudaStream_t st) {
+static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
+  DecodeParams p = p0;
   const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
-  if (lowrank) {
-    k_lowrank_stage1<B><<<p.upr, 256, 0, st>>>(p);
+  const bool csr = p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR);
+  const int n_s1 = lowrank ? (p.r_pad / 32) * ((p.upr + kS1Units - 1) / kS1Units) : 0;
+  const int n_csr = csr ? (p.d.n_out + 255) / 256 : 0;
+  p.has_pre = (n_s1 + n_csr) > 0;
+  const bool pdl = p.has_pre;
+  if (p.has_pre) {
+    const size_t smem = (size_t)kS1Units * kGroup * B * 4;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute((const void*)k_pre<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    k_pre<B><<<n_s1 + n_csr, 256, smem, st>>>(p, n_s1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -610,29 +752,29 @@ static cudaError_t launch_decode_b(const DecodeParams& p, cudaStream_t st) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = lowrank ? 1 : 0;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, k_finish_only<B>, p);
   }
   const int bits = codec_bits(p.d.codec);
   if (p.d.mask == CQL_MASK_2_4) {
-    if (bits == 4) return launch_unit<Unit24<4, B>, B>(p, Unit24<4, B>::kUnitBytes, 0, st, lowrank);
-    return launch_unit<Unit24<3, B>, B>(p, Unit24<3, B>::kUnitBytes, 0, st, lowrank);
+    if (bits == 4) return launch_unit<Unit24<4, B>, B>(p, Unit24<4, B>::kUnitBytes, 0, st, pdl);
+    return launch_unit<Unit24<3, B>, B>(p, Unit24<3, B>::kUnitBytes, 0, st, pdl);
   }
   if (p.d.mask == CQL_MASK_BITMAP50) {
     const int extra = (kDecNT / 32) * UnitBitmap<4, B>::kWinWords * 32 * 4;
-    if (bits == 4) return launch_unit<UnitBitmap<4, B>, B>(p, UnitBitmap<4, B>::kUnitBytes, extra, st, lowrank);
-    return launch_unit<UnitBitmap<3, B>, B>(p, UnitBitmap<3, B>::kUnitBytes, extra, st, lowrank);
+    if (bits == 4) return launch_unit<UnitBitmap<4, B>, B>(p, UnitBitmap<4, B>::kUnitBytes, extra, st, pdl);
+    return launch_unit<UnitBitmap<3, B>, B>(p, UnitBitmap<3, B>::kUnitBytes, extra, st, pdl);
   }
   const int lut_extra = (kDecNT / 32) * 16 * 32 * 4;
   switch (p.d.codec) {
     case CQL_CODEC_INT4_SYM:
-      return launch_unit<UnitDense<4, false, B>, B>(p, UnitDense<4, false, B>::kUnitBytes, 0, st, lowrank);
+      return launch_unit<UnitDense<4, false, B>, B>(p, UnitDense<4, false, B>::kUnitBytes, 0, st, pdl);
     case CQL_CODEC_INT3_SYM:
-      return launch_unit<UnitDense<3, false, B>, B>(p, UnitDense<3, false, B>::kUnitBytes, 0, st, lowrank);
+      return launch_unit<UnitDense<3, false, B>, B>(p, UnitDense<3, false, B>::kUnitBytes, 0, st, pdl);
     case CQL_CODEC_LUT3_ROW:
-      return launch_unit<UnitDense<3, true, B>, B>(p, UnitDense<3, true, B>::kUnitBytes, lut_extra, st, lowrank);
+      return launch_unit<UnitDense<3, true, B>, B>(p, UnitDense<3, true, B>::kUnitBytes, lut_extra, st, pdl);
     default:
-      return launch_unit<UnitDense<4, true, B>, B>(p, UnitDense<4, true, B>::kUnitBytes, lut_extra, st, lowrank);
+      return launch_unit<UnitDense<4, true, B>, B>(p, UnitDense<4, true, B>::kUnitBytes, lut_extra, st, pdl);
   }
 }
 

@@ -82,6 +82,7 @@ struct DecodeParams {
   int n_tiles;
   uint64_t n_units;  // n_rb * upr
   int r_pad;         // rank rounded up to 32
+  int has_pre;       // a pre-kernel (adapter stage 1 and/or CSR rows) runs first, PDL-overlapped
   // workspace
   uint32_t* err;         // [2]
   uint32_t* t_counter;   // [1]   low-rank stage-1 arrival counter
@@ -97,5 +98,17 @@ struct ForwardWorkspace {
 ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch);
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+// Prefill scratch (inside the forward workspace): byte offsets.
+struct PrefillLayout {
+  int r3;          // adapter extension columns (3 r rounded up to 64)
+  int rrows;       // R rows padded to 128
+  int r_pad;       // rank rounded up to 32
+  int ldq;         // K + r3
+  uint64_t qbf, wsc, rbf, rsc, tacc, t3, total;
+};
+PrefillLayout prefill_layout(const cql_desc& d, int m);
+bool prefill_supported(const cql_desc& d, int x_dt);
+cudaError_t launch_prefill(const DecodeParams& p, uint8_t* prefill_ws, cudaStream_t st);
 
 }  // namespace cql

@@ -43,7 +43,7 @@ constexpr int PF_STAGES = 4;
 constexpr int PF_THREADS = 384;
 constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;
 constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;
-constexpr uint32_t PF_WAIT_LIMIT = 1u << 26;
+constexpr uint64_t PF_WAIT_NS = 2000000000ull;   // a wait longer than 2 s is an error
 
 struct PfGemmParams {
   const float* scales;       // [rows][G] fp32
@@ -58,6 +58,7 @@ struct PfGemmParams {
   int out_dt;
   int ldo;                   // leading dimension of out (elements)
   int valid_rows;            // rows that produce output (N, or rank for the T pass)
+  uint32_t idesc;            // tcgen05 instruction descriptor (operand dtype)
   uint32_t* err;
 };
 
@@ -75,10 +76,17 @@ CQL_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 CQL_DEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Bounded wait for the phase of the given parity; false if the limit ran out.
+CQL_DEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase of the given parity to complete, bounded by wall time:
+// false once PF_WAIT_NS has passed (the caller records an error and winds down).
 CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0; it < PF_WAIT_LIMIT; ++it) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -88,8 +96,9 @@ CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    if (it == 0) t0 = globaltimer_ns();
+    else if ((it & 63) == 0 && globaltimer_ns() - t0 > PF_WAIT_NS) return false;
   }
-  return false;
 }
 CQL_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
@@ -126,17 +135,31 @@ CQL_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-CQL_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+#define CQL_R8(v, o) "+f"(v[o]), "+f"(v[o + 1]), "+f"(v[o + 2]), "+f"(v[o + 3]), "+f"(v[o + 4]), "+f"(v[o + 5]), \
+                     "+f"(v[o + 6]), "+f"(v[o + 7])
+// tcgen05.wait::ld, with the loaded registers as in/out operands so that no
+// use of them can be scheduled before the wait.
+CQL_DEV void tmem_wait_ld(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : CQL_R8(v, 0), CQL_R8(v, 8), CQL_R8(v, 16), CQL_R8(v, 24)::"memory");
+}
+// Orders the uses of registers loaded before an earlier tcgen05.wait::ld.
+CQL_DEV void reg_after_wait(float (&v)[32]) {
+  asm volatile("" : CQL_R8(v, 0), CQL_R8(v, 8), CQL_R8(v, 16), CQL_R8(v, 24)::"memory");
+}
+#undef CQL_R8
 
 // Shared-memory matrix descriptor: K-major operand tile written by TMA with
 // 128-byte swizzling (8-row x 128-byte atoms, atoms 1024 bytes apart).
 CQL_DEV uint64_t smem_desc_sw128(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
-// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major,
-// M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PF_BN >> 3) << 17) |
-                            ((uint32_t)(PF_BM >> 4) << 24);
+// Instruction descriptor: kind::f16, A and B both bf16 (format 1) or both fp16
+// (format 0), D = f32, both K-major, M = 128, N = 256.
+CQL_HD uint32_t pf_idesc(bool f16) {
+  const uint32_t fmt = f16 ? 0u : 1u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(PF_BN >> 3) << 17) | ((uint32_t)(PF_BM >> 4) << 24);
+}
 
 // ---------------------------------------------------------------------------
 // the GEMM
@@ -180,9 +203,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const int n_items = p.row_tiles * p.tok_tiles * p.k_splits;
   const int main_blocks = 2 * p.groups;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  // Register split: the launch gives every thread 168 registers; warpgroup 0
+  // (producer, MMA, two idle warps) drops to 40, the two epilogue warpgroups
+  // rise to 232: 128 * 40 + 256 * 232 = 384 * 168.
+  if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    if (warp == 0) {
+    // ---------------- TMA producer ----------------
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -206,9 +233,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 10);
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
     if (lane == 0) {
       uint32_t it = 0, gc = 0;
       bool ok = true;
@@ -231,7 +257,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const uint64_t db = smem_desc_sw128(smem_u32(S.b[s]));
 #pragma unroll
             for (int kk = 0; kk < PF_BK / 16; ++kk)
-              tc_mma(d, da + 2 * kk, db + 2 * kk, kIdesc, (j > 0 || kk > 0) ? 1u : 0u);
+              tc_mma(d, da + 2 * kk, db + 2 * kk, p.idesc, (j > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&S.empty[s]);
           }
           tc_commit(&S.tfull[buf]);
@@ -239,9 +265,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 11);
     }
-  } else if (warp >= 4) {
-    // ---------------- epilogue ----------------
+    }
+  } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    // ---------------- epilogue ----------------
     const int q = warp & 3, h = (warp - 4) >> 2;
     uint32_t gc = 0;
     bool ok = true;
@@ -260,7 +287,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int gn = g0 + g + 1;
         s_next = (g + 1 < g1 - g0) ? __ldg(p.scales + (uint64_t)row * p.groups + gn) : 1.0f;
         const uint32_t buf = gc & 1;
-        if (!mbar_wait(&S.tfull[buf], (gc >> 1) & 1)) { ok = false; break; }
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.tfull[buf], (gc >> 1) & 1));   // warp-uniform
+        if (!ok) break;
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + buf * PF_BN + h * 128;
 #pragma unroll
@@ -268,7 +296,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           float v0[32], v1[32];
           tmem_ld32(base + c * 32, v0);
           tmem_ld32(base + (c + 1) * 32, v1);
-          tmem_wait_ld();
+          tmem_wait_ld(v0);
+          reg_after_wait(v1);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             acc[c * 32 + i] = fmaf(s, v0[i], acc[c * 32 + i]);
@@ -283,36 +312,79 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       if (row < p.valid_rows) {
         const int t0 = tt * PF_BN + h * 128;
         if (p.mode == 0) {
-#pragma unroll 4
+#pragma unroll
           for (int i = 0; i < 128; ++i)
             if (t0 + i < p.m) store_out(p.out, p.out_dt, (uint64_t)(t0 + i) * p.ldo + row, acc[i]);
         } else {
           float* o = reinterpret_cast<float*>(p.out);
-#pragma unroll 4
+#pragma unroll
           for (int i = 0; i < 128; ++i)
             if (t0 + i < p.m) atomicAdd(o + (uint64_t)(t0 + i) * p.ldo + row, acc[i]);
         }
       }
     }
     if (!ok && lane == 0) set_error(p.err, CQL_ERR_TIMEOUT, 12);
-  } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
 }
 
 // ---------------------------------------------------------------------------
 // dequantisation to exact bf16 codes (+ scales), adapters as hi/lo splits
 // ---------------------------------------------------------------------------
 CQL_DEV uint16_t bf16_bits_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
-CQL_DEV uint16_t int_to_bf16(int q) { return bf16_bits_rn((float)q); }   // exact for |q| <= 256
+// 16-bit operand encodings (bf16 unless f16): round to nearest even, and back.
+CQL_DEV uint16_t to16(float v, int f16) { return f16 ? __half_as_ushort(__float2half_rn(v)) : bf16_bits_rn(v); }
+CQL_DEV float from16(uint16_t b, int f16) { return f16 ? f16_bits_to_f32(b) : bf16_bits_to_f32(b); }
+CQL_DEV uint16_t int_to16(int q, int f16) { return to16((float)q, f16); }   // exact for |q| <= 256
 
-// One thread per (row, 128-column unit) of W: q codes -> bf16, zeros where the
-// 2:4 mask pruned; and the unit's scale as fp32.
-__global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* scales) {
+// 2:4 int4 unit of one row -> 128 codes as 16-bit operands (zeros where
+// pruned): one 16-byte load of pattern nibbles, two of codes.
+__global__ void k_pf_dequant_w24(DecodeParams p, uint16_t* qbf, int ldq, float* scales, int f16) {
+  const int G = p.upr;
+  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (uint64_t)p.d.n_out * G) return;
+  const int g = (int)(id / p.d.n_out), n = (int)(id % p.d.n_out);   // consecutive threads: consecutive rows
+  const int rb = n >> 5, lane = n & 31;
+  const uint4 va = ldg_stream(p.values + slab_off(rb, 2 * g, p.rb.values) + lane * 16);
+  const uint4 vb = ldg_stream(p.values + slab_off(rb, 2 * g + 1, p.rb.values) + lane * 16);
+  const uint4 mm = ldg_stream(p.meta + slab_off(rb, g, p.rb.meta) + lane * 16);
+  const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+  const uint32_t mw[4] = {mm.x, mm.y, mm.z, mm.w};
+  uint4* dst = reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + (uint64_t)g * 128);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {             // 8 columns = 2 groups per 16-byte store
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int gi = 2 * c + h;
+      const uint32_t pt = (mw[gi >> 3] >> (4 * (gi & 7))) & 15u;
+      const uint32_t byte = (vw[gi >> 2] >> (8 * (gi & 3))) & 0xFFu;
+      const uint32_t q0 = int_to16((int)(byte & 15u) - 8, f16), q1 = int_to16((int)(byte >> 4) - 8, f16);
+      uint32_t lo = 0, hi = 0;               // columns (0,1) and (2,3) of the group
+      switch (pt) {
+        case 0: lo = q0 | (q1 << 16); break;                 // (0,1)
+        case 1: lo = q0; hi = q1; break;                     // (0,2)
+        case 2: lo = q0; hi = q1 << 16; break;               // (0,3)
+        case 3: lo = q0 << 16; hi = q1; break;               // (1,2)
+        case 4: lo = q0 << 16; hi = q1 << 16; break;         // (1,3)
+        default: hi = q0 | (q1 << 16); break;                // (2,3)
+      }
+      w[2 * h] = lo;
+      w[2 * h + 1] = hi;
+    }
+    dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  scales[(uint64_t)n * G + g] = f16_bits_to_f32(ldg_u16(p.scales + rit(n, 2 * g, p.rb.scales)));
+}
+
+// Any uniform codec with the 2:4 mask or no mask (generic bit extraction).
+__global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* scales, int f16) {
   const int G = p.upr;
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= (uint64_t)p.d.n_out * G) return;
@@ -340,8 +412,8 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
         qv[h] = (int)(c & mask) - bias;
       }
       for (int i = 0; i < 4; ++i) outv[4 * gi + i] = 0;
-      outv[4 * gi + i0] = int_to_bf16(qv[0]);
-      outv[4 * gi + i1] = int_to_bf16(qv[1]);
+      outv[4 * gi + i0] = int_to16(qv[0], f16);
+      outv[4 * gi + i1] = int_to16(qv[1], f16);
     }
   } else {
     const uint64_t bit0 = (uint64_t)128 * bits * g;
@@ -352,7 +424,7 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
         const uint64_t sb = bp + t;
         code |= ((uint32_t)(p.values[rit(n, sb >> 3, p.rb.values)] >> (sb & 7)) & 1u) << t;
       }
-      outv[c] = int_to_bf16((int)code - bias);
+      outv[c] = int_to16((int)code - bias, f16);
     }
   }
   uint4* dst = reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + (uint64_t)g * 128);
@@ -369,7 +441,7 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
 
 // Adapter columns of the main operand: [Lhi | Lhi | Llo | 0] at columns
 // K .. K + r3 of row n, with L^ = q_L s_L exact in fp32 and Lhi + Llo = L^.
-__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3) {
+__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3, int f16) {
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int r = p.d.rank;
   if (id >= (uint64_t)p.d.n_out * r3) return;
@@ -381,14 +453,14 @@ __global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3) {
     const int q = (int)((byte >> (4 * (j & 1))) & 15u) - 8;
     const float s = f16_bits_to_f32(p.l_scales[(uint64_t)(n / kGroup) * r + j]);
     const float l = (float)q * s;                            // exact (<= 14 significant bits)
-    const uint16_t hi = bf16_bits_rn(l);
-    v = part < 2 ? hi : bf16_bits_rn(l - bf16_bits_to_f32(hi));
+    const uint16_t hi = to16(l, f16);
+    v = part < 2 ? hi : to16(l - from16(hi, f16), f16);
   }
   qbf[(uint64_t)n * ldq + p.d.k_in + c] = v;
 }
 
 // R rows (padded to 128) as bf16 codes and fp32 scales.
-__global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, int rows) {
+__global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, int rows, int f16) {
   const int K = p.d.k_in, G = p.upr;
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= (uint64_t)rows * K) return;
@@ -396,7 +468,7 @@ __global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, in
   uint16_t v = 0;
   if (j < p.d.rank) {
     const uint32_t byte = p.r_values[rit(j, k / 2, p.rb.r_values)];
-    v = int_to_bf16((int)((byte >> (4 * (k & 1))) & 15u) - 8);
+    v = int_to16((int)((byte >> (4 * (k & 1))) & 15u) - 8, f16);
   }
   rbf[id] = v;
   if (k % kGroup == 0)
@@ -405,8 +477,8 @@ __global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, in
                      : 0.0f;
 }
 
-// T [m][r_pad] fp32 -> [Thi | Tlo | Thi | 0] bf16 [m][r3]; clears T.
-__global__ void k_pf_tsplit(float* t, int ldt, uint16_t* t3, int r3, int r, int m) {
+// T [m][r_pad] fp32 -> [Thi | Tlo | Thi | 0] as bf16 (or fp16) [m][r3].
+__global__ void k_pf_tsplit(const float* t, int ldt, uint16_t* t3, int r3, int r, int m, int f16) {
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= (uint64_t)m * r3) return;
   const int row = (int)(id / r3), c = (int)(id % r3);
@@ -414,12 +486,10 @@ __global__ void k_pf_tsplit(float* t, int ldt, uint16_t* t3, int r3, int r, int 
   if (c < 3 * r) {
     const int j = c % r, part = c / r;                       // 0: hi, 1: lo, 2: hi
     const float x = t[(uint64_t)row * ldt + j];
-    const uint16_t hi = bf16_bits_rn(x);
-    v = part == 1 ? bf16_bits_rn(x - bf16_bits_to_f32(hi)) : hi;
+    const uint16_t hi = to16(x, f16);
+    v = part == 1 ? to16(x - from16(hi, f16), f16) : hi;
   }
   t3[id] = v;
-  __syncthreads();
-  if (c < r && c < ldt) t[(uint64_t)row * ldt + c] = 0.0f;   // thread (row, c) read (row, c % r) only for c < 3r
 }
 
 // ---------------------------------------------------------------------------
@@ -476,9 +546,29 @@ static int sm_count_pf() {
   return v > 0 ? v : 148;
 }
 
+bool prefill_supported(const cql_desc& d, int x_dt) {
+  if (codec_is_lut(d.codec) || d.mask == CQL_MASK_BITMAP50) return false;
+  if (d.outlier_frac > 0.0f) return false;
+  return x_dt == CQL_DT_BF16 || x_dt == CQL_DT_F16;
+}
+
+// The epilogue raises its register budget with setmaxnreg; that only works if
+// the kernel was compiled to the full 168 registers per thread of a 384-thread
+// block (128 * 40 + 256 * 232 == 384 * 168).  Checked once before launching.
+static cudaError_t check_gemm_regs() {
+  static int ok = -1;
+  if (ok < 0) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, (const void*)k_pf_gemm) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+    ok = a.numRegs == 168 ? 1 : 0;
+  }
+  return ok ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st) {
   const PrefillLayout L = prefill_layout(p.d, p.batch);
   const int N = p.d.n_out, K = p.d.k_in, r = p.d.rank, m = p.batch, G = p.upr;
+  const int f16 = p.xdt == CQL_DT_F16 ? 1 : 0;
   uint16_t* qbf = reinterpret_cast<uint16_t*>(pws + L.qbf);
   float* wsc = reinterpret_cast<float*>(pws + L.wsc);
   uint16_t* rbf = reinterpret_cast<uint16_t*>(pws + L.rbf);
@@ -487,41 +577,48 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   uint16_t* t3 = reinterpret_cast<uint16_t*>(pws + L.t3);
   const bool lowrank = r > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
   const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
+  cudaError_t e = check_gemm_regs();
+  if (e != cudaSuccess) return e;
 
   static bool attr_set = false;
   const size_t smem = sizeof(PfSmem) + 1024;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute((const void*)k_pf_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute((const void*)k_pf_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const uint64_t nw = (uint64_t)N * G;
-  k_pf_dequant_w<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc);
+  if (p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM)
+    k_pf_dequant_w24<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc, f16);
+  else
+    k_pf_dequant_w<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc, f16);
   if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);       // main term off: zero scales
   if (lowrank) {
     const uint64_t nl = (uint64_t)N * L.r3;
-    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.r3);
+    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.r3, f16);
     const uint64_t nr = (uint64_t)L.rrows * K;
-    k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows);
+    k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows, f16);
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int sms = sm_count_pf();
+  const uint32_t idesc = pf_idesc(f16 != 0);
   CUtensorMap mA, mB, mT, mR;
   if (!make_map(&mB, p.x, (uint64_t)m, (uint64_t)K, (uint64_t)K, PF_BN)) return cudaErrorInvalidValue;
   if (lowrank) {
-    // T pass: T = X R^T, split over K, fp32 atomics into tacc (zero on entry)
+    // T pass: T = X R^T, split over K, fp32 atomics into tacc
+    if ((e = cudaMemsetAsync(tacc, 0, (uint64_t)m * L.r_pad * 4, st)) != cudaSuccess) return e;
     if (!make_map(&mR, rbf, (uint64_t)L.rrows, (uint64_t)K, (uint64_t)K, PF_BM)) return cudaErrorInvalidValue;
     PfGemmParams t{};
     t.scales = rsc; t.rows = L.rrows; t.m = m; t.groups = G; t.lr_blocks = 0;
     t.row_tiles = L.rrows / PF_BM; t.tok_tiles = (m + PF_BN - 1) / PF_BN;
     const int tiles = t.row_tiles * t.tok_tiles;
     t.k_splits = max(1, min(G, sms / max(tiles, 1)));
-    t.mode = 1; t.out = tacc; t.out_dt = CQL_DT_F32; t.ldo = L.r_pad; t.valid_rows = r; t.err = p.err;
+    t.mode = 1; t.out = tacc; t.out_dt = CQL_DT_F32; t.ldo = L.r_pad; t.valid_rows = r; t.idesc = idesc;
+    t.err = p.err;
     const int items = tiles * t.k_splits;
     k_pf_gemm<<<min(items, sms), PF_THREADS, smem, st>>>(mR, mB, mB, t);
     const uint64_t nt = (uint64_t)m * L.r3;
-    k_pf_tsplit<<<(unsigned)((nt + 255) / 256), 256, 0, st>>>(tacc, L.r_pad, t3, L.r3, r, m);
+    k_pf_tsplit<<<(unsigned)((nt + 255) / 256), 256, 0, st>>>(tacc, L.r_pad, t3, L.r3, r, m, f16);
     if (!make_map(&mT, t3, (uint64_t)m, (uint64_t)L.r3, (uint64_t)L.r3, PF_BN)) return cudaErrorInvalidValue;
   } else {
     mT = mB;
@@ -530,7 +627,7 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   PfGemmParams g{};
   g.scales = wsc; g.rows = N; g.m = m; g.groups = G; g.lr_blocks = lowrank ? L.r3 / PF_BK : 0;
   g.row_tiles = N / PF_BM; g.tok_tiles = (m + PF_BN - 1) / PF_BN; g.k_splits = 1;
-  g.mode = 0; g.out = p.y; g.out_dt = p.ydt; g.ldo = N; g.valid_rows = N; g.err = p.err;
+  g.mode = 0; g.out = p.y; g.out_dt = p.ydt; g.ldo = N; g.valid_rows = N; g.idesc = idesc; g.err = p.err;
   const int items = g.row_tiles * g.tok_tiles;
   k_pf_gemm<<<min(items, sms), PF_THREADS, smem, st>>>(mA, mB, mT, g);
   return cudaGetLastError();
