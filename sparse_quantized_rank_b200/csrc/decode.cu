@@ -5,7 +5,8 @@
 //  * lanes = rows.  A warp owns a block of 32 output rows and walks K in
 //    units of 128 columns (one scale group).  The packed planes are row
 //    interleaved, so at every step the 32 lanes read 16 consecutive bytes
-//    each: one fully coalesced 512-byte access per warp per slab.
+//    each: one fully coalesced 512-byte access per warp per slab, staged into
+//    a per-warp ring of shared memory with cp.async, 4 units in flight.
 //  * Because all lanes of a warp sit on the same columns, the activations are
 //    warp-uniform.  For the 2:4 mask the x pair a kept pair multiplies,
 //    (x[4g+i0], x[4g+i1]), is read from a shared-memory table indexed by the
@@ -17,15 +18,18 @@
 //    are packed fp32x2 FMAs.  The group scale multiplies the group's partial
 //    sum once (SLiM-Quant's per-group scale, review summary "SLIM-Quant").
 //  * Work is balanced at unit granularity: the (row block, unit) space is cut
-//    into one contiguous range per CTA (persistent grid over all SMs).  Partial
-//    row sums are added into an fp32 accumulator with reductions at L2; the
-//    warp that completes a row block (arrival counter) runs the epilogue: the
-//    CSR outliers of its rows (SqueezeLLM "Approach": dense-and-sparse), the
-//    second low-rank stage L_q t (SLiM "Low-rank adapter quantization"), the
-//    final rounding, and the reset of the accumulator for the next call.
-//  * The first low-rank stage t = R_q x runs in its own small kernel that
-//    starts the main kernel at once through programmatic dependent launch; the
-//    epilogue waits on it with griddepcontrol.wait, long after it finished.
+//    into one contiguous range per CTA (persistent grid, one CTA per SM), and
+//    each warp takes a contiguous part of it.  Partial row sums are added into
+//    an fp32 accumulator with reductions at L2, with no fence or counter on the
+//    streaming path.
+//  * Three kernels per call, chained by programmatic dependent launch:
+//      k_pre       t = R_q x partial sums (SLiM "Low-rank adapter
+//                  quantization") and the CSR outlier rows added into the
+//                  accumulator (SqueezeLLM "Approach": dense-and-sparse);
+//      k_decode    the main term, streaming;
+//      k_epilogue  y = accumulator + L_q t, rounding, accumulator reset;
+//    each later kernel starts early and waits (griddepcontrol.wait) only where
+//    it reads the earlier kernel's results.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -74,69 +78,13 @@ CQL_DEV void stage_x(const DecodeParams& p, float* xs, int c0, int ncols) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// epilogue for one row block: accumulator + CSR + low rank -> y
-// ---------------------------------------------------------------------------
+// Add a warp's partial row sums into the fp32 accumulator (reductions at L2).
 template <int B>
-CQL_DEV void finish_rowblock(const DecodeParams& p, int rb, int lane) {
-  const int N = p.d.n_out;
-  const int row = rb * 32 + lane;
-  if (p.has_pre) pdl_wait();            // CSR rows and t = R_q x are complete
-  float acc[B];
-#pragma unroll
-  for (int b = 0; b < B; ++b) {
-    acc[b] = 0.0f;
-    if (b < p.batch) {
-      float* a = p.y_acc + (uint64_t)b * N + row;
-      acc[b] = ld_cg_f32(a);
-      *a = 0.0f;
-    }
-  }
-  if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK)) {
-    const int r = p.d.rank, g = row / kGroup;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {             // rank <= 256: at most 8 chunks of 32
-      if (32 * m >= r) break;
-      const int j = 32 * m + lane;
-      float u[B];
-      const float ls = j < r ? f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) : 0.0f;
-#pragma unroll
-      for (int b = 0; b < B; ++b) u[b] = j < r ? ls * ld_cg_f32(p.t_final + (uint64_t)b * p.r_pad + j) : 0.0f;
-      const uint4 w = ldg_stream(p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
-      const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        if (32 * m + jj >= r) break;
-        const float q = (float)((int)((wd[jj >> 3] >> (4 * (jj & 7))) & 15u) - 8);
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[b] = fmaf(q, __shfl_sync(0xffffffffu, u[b], jj), acc[b]);
-      }
-    }
-  }
-#pragma unroll
-  for (int b = 0; b < B; ++b)
-    if (b < p.batch) store_out(p.y, p.ydt, (uint64_t)b * N + row, acc[b]);
-  if (lane == 0) p.counters[rb] = 0u;
-}
-
-// Add a warp's partial sums of a row block and count its units; the warp
-// that completes the row block runs the epilogue.
-template <int B>
-CQL_DEV void flush_rowblock(const DecodeParams& p, int rb, uint32_t units, const float (&acc)[B], int lane) {
-  const int N = p.d.n_out;
+CQL_DEV void red_rows(const DecodeParams& p, int rb, const float (&acc)[B], int lane) {
   const int row = rb * 32 + lane;
 #pragma unroll
   for (int b = 0; b < B; ++b)
-    if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * N + row, acc[b]);
-  __threadfence();
-  __syncwarp();
-  uint32_t old = 0;
-  if (lane == 0) old = atomicAdd(p.counters + rb, units);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (old + units == (uint32_t)p.upr) {
-    __threadfence();
-    finish_rowblock<B>(p, rb, lane);
-  }
+    if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
 }
 
 // ---------------------------------------------------------------------------
@@ -168,17 +116,29 @@ struct Unit24 {
     float* xs = reinterpret_cast<float*>(smem + (size_t)p.ktu * kTableBytes);
     stage_x<B>(p, xs, c0, units * kGroup);
     __syncthreads();
-    for (int i = threadIdx.x; i < ngroups * NBP * 6; i += blockDim.x) {
-      const int pt = i % 6, t2 = i / 6, bp = t2 % NBP, g = t2 / NBP;
-      int i0, i1;
-      pair_of(pt, i0, i1);
-      const float* xc = xs + (4 * g) * B;
+    // one (group, batch pair) per iteration: read its 4 columns once, write
+    // the 6 pattern entries with straight-line stores
+    for (int i = threadIdx.x; i < ngroups * NBP; i += blockDim.x) {
+      const int bp = i % NBP, g = i / NBP;
+      const float* xc = xs + (4 * g) * B + 2 * bp;
       if (B == 1) {
-        *reinterpret_cast<float2*>(smem + g * 64 + pt * 8) = make_float2(xc[i0], xc[i1]);
+        const float4 x4 = *reinterpret_cast<const float4*>(xc);
+        float4* e = reinterpret_cast<float4*>(smem + g * 64);
+        e[0] = make_float4(x4.x, x4.y, x4.x, x4.z);   // patterns 0 (0,1), 1 (0,2)
+        e[1] = make_float4(x4.x, x4.w, x4.y, x4.z);   // patterns 2 (0,3), 3 (1,2)
+        e[2] = make_float4(x4.y, x4.w, x4.z, x4.w);   // patterns 4 (1,3), 5 (2,3)
       } else {
-        const int b = 2 * bp;
-        *reinterpret_cast<float4*>(smem + ((g * NBP + bp) * 8 + pt) * 16) =
-            make_float4(xc[i0 * B + b], xc[i1 * B + b], xc[i0 * B + b + 1], xc[i1 * B + b + 1]);
+        const float2 c0v = *reinterpret_cast<const float2*>(xc);          // column 0, batches b, b+1
+        const float2 c1v = *reinterpret_cast<const float2*>(xc + B);
+        const float2 c2v = *reinterpret_cast<const float2*>(xc + 2 * B);
+        const float2 c3v = *reinterpret_cast<const float2*>(xc + 3 * B);
+        float4* e = reinterpret_cast<float4*>(smem + (g * NBP + bp) * 128);
+        e[0] = make_float4(c0v.x, c1v.x, c0v.y, c1v.y);
+        e[1] = make_float4(c0v.x, c2v.x, c0v.y, c2v.y);
+        e[2] = make_float4(c0v.x, c3v.x, c0v.y, c3v.y);
+        e[3] = make_float4(c1v.x, c2v.x, c1v.y, c2v.y);
+        e[4] = make_float4(c1v.x, c3v.x, c1v.y, c3v.y);
+        e[5] = make_float4(c2v.x, c3v.x, c2v.y, c3v.y);
       }
     }
   }
@@ -475,6 +435,7 @@ template <class U, int B>
 __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(DecodeParams p, int ring_off) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_launch_dependents();                          // let the epilogue kernel get resident
   if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
   // this warp's ring of kDepth unit slots; lane l owns bytes [16 l, 16 l + 16) of every 512-byte slab
   uint8_t* ring = smem + ring_off + (size_t)warp * (kDepth * U::kSlabs * 512) + lane * 16;
@@ -486,33 +447,36 @@ __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(Decode
     unit_coords(p, u, kt, rb, ut);
     const uint64_t tnext = tile_begin(p, kt + 1);
     const uint64_t tend = uend < tnext ? uend : tnext;
+    const uint64_t n = tend - u;
+    const uint64_t wb = u + n * warp / kDecNW, we = u + n * (warp + 1) / kDecNW;
+    const int ts = tile_size(p, kt);
+    const int uk0 = kt * p.ktu;
+    int cur_rb = 0, cur_ut = 0;
+    if (wb < we) {
+      int kt0;
+      unit_coords(p, wb, kt0, cur_rb, cur_ut);
+    }
+    // prologue: start streaming this warp's first kDepth units before the
+    // tile's tables are built (the copies do not depend on them)
+    int irb = cur_rb, iut = cur_ut;
+    uint32_t sc[kDepth];
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      sc[d] = 0;
+      if (wb + d < we) {
+        sc[d] = U::issue(p, irb, uk0 + iut, lane, ring + d * (U::kSlabs * 512));
+        if (++iut == ts) { iut = 0; ++irb; }
+      }
+      cp_async_commit();
+    }
     __syncthreads();
     U::build(p, smem, kt);
     __syncthreads();
-    const uint64_t n = tend - u;
-    const uint64_t wb = u + n * warp / kDecNW, we = u + n * (warp + 1) / kDecNW;
     if (wb < we) {
-      int kt0, cur_rb, cur_ut;
-      unit_coords(p, wb, kt0, cur_rb, cur_ut);
-      const int ts = tile_size(p, kt);
-      const int uk0 = kt * p.ktu;
-      // prologue: stage the first kDepth units
-      int irb = cur_rb, iut = cur_ut;
-      uint32_t sc[kDepth];
-#pragma unroll
-      for (int d = 0; d < kDepth; ++d) {
-        sc[d] = 0;
-        if (wb + d < we) {
-          sc[d] = U::issue(p, irb, uk0 + iut, lane, ring + d * (U::kSlabs * 512));
-          if (++iut == ts) { iut = 0; ++irb; }
-        }
-        cp_async_commit();
-      }
       U::on_row(p, smem, cur_rb, lane);
       float acc[B];
 #pragma unroll
       for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-      uint32_t cnt = 0;
       int slot = 0;
       for (uint64_t i = wb; i < we; ++i) {
         uint8_t* sl = ring + slot * (U::kSlabs * 512);
@@ -530,15 +494,13 @@ __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(Decode
         cp_async_commit();
         if (++slot == kDepth) slot = 0;
         Call<U, B>::compute(p, smem, f, cur_ut, lane, cur_rb, acc);
-        ++cnt;
         int nrb = cur_rb, nut = cur_ut + 1;
         if (nut == ts) { nut = 0; ++nrb; }
         const bool more = i + 1 < we;
         if (!more || nrb != cur_rb) {
-          flush_rowblock<B>(p, cur_rb, cnt, acc, lane);
+          red_rows<B>(p, cur_rb, acc, lane);
 #pragma unroll
           for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-          cnt = 0;
           if (more) U::on_row(p, smem, nrb, lane);
         }
         cur_rb = nrb;
@@ -548,16 +510,78 @@ __global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(Decode
     cp_async_wait<0>();
     u = tend;
   }
+  // complete only after the pre-kernel: the epilogue, which waits on this
+  // grid, then also sees the pre-kernel's CSR sums and adapter partials
+  if (p.has_pre && threadIdx.x == 0) pdl_wait();
 }
 
-// Epilogue only (main term disabled by CQL_FLAG_NO_MAIN): a warp per row block.
+// ---------------------------------------------------------------------------
+// epilogue: a warp per row block (lanes = rows).
+//   y = accumulator + deq(L_q) t,  t = sum of the pre-kernel's slices,
+// rounded to the output dtype; the accumulator is left zeroed.  The packed L
+// codes and scales are read before waiting on the previous kernel; the
+// accumulator and t only after.
+// ---------------------------------------------------------------------------
 template <int B>
-__global__ void __launch_bounds__(256, 1) k_finish_only(DecodeParams p) {
+__global__ void __launch_bounds__(256, 1) k_epilogue(DecodeParams p, int kq) {
   const int lane = threadIdx.x & 31;
   const int rb = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
-  if (rb >= p.n_rb) return;
-  finish_rowblock<B>(p, rb, lane);
+  const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
+  if (rb >= p.n_rb) {
+    pdl_wait();
+    return;
+  }
+  const int N = p.d.n_out, r = p.d.rank;
+  const int row = rb * 32 + lane, g = row / kGroup;
+  uint4 lv[8];
+  float ls[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {                     // rank <= 256: at most 8 chunks of 32
+    lv[m] = make_uint4(0u, 0u, 0u, 0u);
+    ls[m] = 0.0f;
+    if (lowrank && 32 * m < r) {
+      lv[m] = ldg_stream(p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
+      const int j = 32 * m + lane;
+      ls[m] = j < r ? f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) : 0.0f;
+    }
+  }
+  pdl_wait();                                       // main term (and pre-kernel) complete
+  float acc[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    acc[b] = 0.0f;
+    if (b < p.batch) {
+      float* a = p.y_acc + (uint64_t)b * N + row;
+      acc[b] = ld_cg_f32(a);
+      *a = 0.0f;
+    }
+  }
+  if (lowrank) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      if (32 * m >= r) break;
+      const int j = 32 * m + lane;
+      float u[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float t = 0.0f;
+        if (j < r)
+          for (int k = 0; k < kq; ++k) t += ld_cg_f32(p.t_part + ((uint64_t)k * B + b) * p.r_pad + j);
+        u[b] = ls[m] * t;
+      }
+      const uint32_t wd[4] = {lv[m].x, lv[m].y, lv[m].z, lv[m].w};
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        if (32 * m + jj >= r) break;
+        const float q = (float)((int)((wd[jj >> 3] >> (4 * (jj & 7))) & 15u) - 8);
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[b] = fmaf(q, __shfl_sync(0xffffffffu, u[b], jj), acc[b]);
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+    if (b < p.batch) store_out(p.y, p.ydt, (uint64_t)b * N + row, acc[b]);
 }
 
 // ---------------------------------------------------------------------------
@@ -569,8 +593,8 @@ __global__ void __launch_bounds__(256, 1) k_finish_only(DecodeParams p) {
 //  * blocks [n_s1, ..): the CSR outliers, a thread per output row, added into
 //    the fp32 accumulator (SqueezeLLM "Approach": the sparse part of the
 //    dense-and-sparse decomposition).
-// The decode kernel's epilogue waits for this grid (griddepcontrol.wait)
-// before it reads the accumulator or t_final.
+// The epilogue kernel reads these results only after griddepcontrol.wait
+// (the main kernel completes only after this grid).
 // ---------------------------------------------------------------------------
 constexpr int kS1Units = 8;
 
@@ -578,24 +602,27 @@ template <int B>
 __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
   pdl_launch_dependents();
   extern __shared__ __align__(16) float s1[];
-  __shared__ bool s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (blockIdx.x < n_s1) {
     const int KQ = (p.upr + kS1Units - 1) / kS1Units;
     const int rbR = blockIdx.x / KQ, kq = blockIdx.x % KQ;
     const int u0 = kq * kS1Units, u1 = min(p.upr, u0 + kS1Units);
+    const int j = 32 * rbR + lane;
+    const int u = u0 + warp;                          // one unit per warp (kS1Units == 8 warps)
+    uint4 q4[4];
+    float sc = 0.0f;
+    if (u < u1) {                                     // R codes first: they do not depend on x
+      const uint8_t* base = p.r_values + slab_off(rbR, 4 * u, p.rb.r_values) + lane * 16;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) q4[s] = ldg_stream(base + 512 * s);
+      sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit(j, 2 * u, p.rb.r_scales)));
+    }
     stage_x<B>(p, s1, u0 * kGroup, (u1 - u0) * kGroup);
     __syncthreads();
     float acc[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-    const int j = 32 * rbR + lane;
-    for (int u = u0 + warp; u < u1; u += 8) {
-      const uint8_t* base = p.r_values + slab_off(rbR, 4 * u, p.rb.r_values) + lane * 16;
-      uint4 q4[4];
-#pragma unroll
-      for (int s = 0; s < 4; ++s) q4[s] = ldg_stream(base + 512 * s);
-      const float sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit(j, 2 * u, p.rb.r_scales)));
+    if (u < u1) {
       const float* xs = s1 + (u - u0) * kGroup * B;
       float au[B];
 #pragma unroll
@@ -611,7 +638,7 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
         }
       }
 #pragma unroll
-      for (int b = 0; b < B; ++b) acc[b] = fmaf(sc, au[b], acc[b]);
+      for (int b = 0; b < B; ++b) acc[b] = sc * au[b];
     }
     __syncthreads();                                   // x no longer needed: reuse for partials
 #pragma unroll
@@ -623,21 +650,6 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
 #pragma unroll
       for (int w = 0; w < 8; ++w) t += s1[(w * B + b) * 32 + l];
       p.t_part[((uint64_t)kq * B + b) * p.r_pad + 32 * rbR + l] = t;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(p.t_counter, 1u) == (uint32_t)n_s1 - 1;
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      for (int i = threadIdx.x; i < B * p.r_pad; i += blockDim.x) {
-        const int b = i / p.r_pad, jj = i - b * p.r_pad;
-        float t = 0.0f;
-#pragma unroll 4
-        for (int k2 = 0; k2 < KQ; ++k2) t += ld_cg_f32(p.t_part + ((uint64_t)k2 * B + b) * p.r_pad + jj);
-        p.t_final[(uint64_t)b * p.r_pad + jj] = t;
-      }
-      if (threadIdx.x == 0) *p.t_counter = 0u;
     }
   } else {
     const int row = (blockIdx.x - n_s1) * blockDim.x + threadIdx.x;
@@ -720,52 +732,34 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
   return cudaLaunchKernelEx(&cfg, k_decode<U, B>, p, ring_off);
 }
 
+static cudaError_t launch_pdl(const void* f, void** args, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelExC(&cfg, f, args);
+}
+
 template <int B>
-static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
-  DecodeParams p = p0;
-  const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
-  const bool csr = p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR);
-  const int n_s1 = lowrank ? (p.r_pad / 32) * ((p.upr + kS1Units - 1) / kS1Units) : 0;
-  const int n_csr = csr ? (p.d.n_out + 255) / 256 : 0;
-  p.has_pre = (n_s1 + n_csr) > 0;
-  const bool pdl = p.has_pre;
-  if (p.has_pre) {
-    const size_t smem = (size_t)kS1Units * kGroup * B * 4;
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute((const void*)k_pre<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
-    k_pre<B><<<n_s1 + n_csr, 256, smem, st>>>(p, n_s1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if (p.flags & CQL_FLAG_NO_MAIN) {
-    const int blocks = (p.n_rb * 32 + 255) / 256;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(256);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_finish_only<B>, p);
-  }
+static cudaError_t launch_main(const DecodeParams& p, cudaStream_t st, bool pdl) {
   const int bits = codec_bits(p.d.codec);
   if (p.d.mask == CQL_MASK_2_4) {
     if (bits == 4) return launch_unit<Unit24<4, B>, B>(p, Unit24<4, B>::kUnitBytes, 0, st, pdl);
     return launch_unit<Unit24<3, B>, B>(p, Unit24<3, B>::kUnitBytes, 0, st, pdl);
   }
   if (p.d.mask == CQL_MASK_BITMAP50) {
-    const int extra = (kDecNT / 32) * UnitBitmap<4, B>::kWinWords * 32 * 4;
+    const int extra = kDecNW * UnitBitmap<4, B>::kWinWords * 32 * 4;
     if (bits == 4) return launch_unit<UnitBitmap<4, B>, B>(p, UnitBitmap<4, B>::kUnitBytes, extra, st, pdl);
     return launch_unit<UnitBitmap<3, B>, B>(p, UnitBitmap<3, B>::kUnitBytes, extra, st, pdl);
   }
-  const int lut_extra = (kDecNT / 32) * 16 * 32 * 4;
+  const int lut_extra = kDecNW * 16 * 32 * 4;
   switch (p.d.codec) {
     case CQL_CODEC_INT4_SYM:
       return launch_unit<UnitDense<4, false, B>, B>(p, UnitDense<4, false, B>::kUnitBytes, 0, st, pdl);
@@ -776,6 +770,39 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
     default:
       return launch_unit<UnitDense<4, true, B>, B>(p, UnitDense<4, true, B>::kUnitBytes, lut_extra, st, pdl);
   }
+}
+
+// pre (adapter partials, CSR rows) -> main term -> epilogue, each PDL-chained
+// to the one before it.
+template <int B>
+static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
+  DecodeParams p = p0;
+  const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
+  const bool csr = p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR);
+  const int kq = (p.upr + kS1Units - 1) / kS1Units;
+  const int n_s1 = lowrank ? (p.r_pad / 32) * kq : 0;
+  const int n_csr = csr ? (p.d.n_out + 255) / 256 : 0;
+  p.has_pre = (n_s1 + n_csr) > 0;
+  cudaError_t e;
+  if (p.has_pre) {
+    const size_t smem = (size_t)kS1Units * kGroup * B * 4;
+    static bool attr_set = false;
+    if (!attr_set) {
+      e = cudaFuncSetAttribute((const void*)k_pre<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    k_pre<B><<<n_s1 + n_csr, 256, smem, st>>>(p, n_s1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
+  if (main_on) {
+    if ((e = launch_main<B>(p, st, p.has_pre)) != cudaSuccess) return e;
+  }
+  int kq_arg = kq;
+  void* args[2] = {&p, &kq_arg};
+  const dim3 grid((p.n_rb * 32 + 255) / 256);
+  return launch_pdl((const void*)k_epilogue<B>, args, grid, dim3(256), 0, st, main_on || p.has_pre);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st) {

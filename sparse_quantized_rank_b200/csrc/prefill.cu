@@ -343,44 +343,48 @@ CQL_DEV uint16_t to16(float v, int f16) { return f16 ? __half_as_ushort(__float2
 CQL_DEV float from16(uint16_t b, int f16) { return f16 ? f16_bits_to_f32(b) : bf16_bits_to_f32(b); }
 CQL_DEV uint16_t int_to16(int q, int f16) { return to16((float)q, f16); }   // exact for |q| <= 256
 
-// 2:4 int4 unit of one row -> 128 codes as 16-bit operands (zeros where
-// pruned): one 16-byte load of pattern nibbles, two of codes.
-__global__ void k_pf_dequant_w24(DecodeParams p, uint16_t* qbf, int ldq, float* scales, int f16) {
+// 2:4 int4 -> 16-bit codes, zeros where pruned.  A warp per (row block,
+// 128-column unit): coalesced 16-byte loads of its code and pattern slabs
+// (lane = row), branch-free expansion of each group, a transpose through
+// shared memory, then full-row 16-byte stores (two rows per instruction).
+constexpr int kDqWarps = 4;
+__global__ void __launch_bounds__(kDqWarps * 32) k_pf_dequant_w24(DecodeParams p, uint16_t* qbf, int ldq,
+                                                                  float* scales, int f16) {
+  __shared__ uint4 stage[kDqWarps][32][17];          // 17: pad against bank conflicts
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = p.upr;
-  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= (uint64_t)p.d.n_out * G) return;
-  const int g = (int)(id / p.d.n_out), n = (int)(id % p.d.n_out);   // consecutive threads: consecutive rows
-  const int rb = n >> 5, lane = n & 31;
+  const uint64_t wid = (uint64_t)blockIdx.x * kDqWarps + warp;
+  if (wid >= (uint64_t)p.n_rb * G) return;
+  const int rb = (int)(wid / G), g = (int)(wid % G);
   const uint4 va = ldg_stream(p.values + slab_off(rb, 2 * g, p.rb.values) + lane * 16);
   const uint4 vb = ldg_stream(p.values + slab_off(rb, 2 * g + 1, p.rb.values) + lane * 16);
   const uint4 mm = ldg_stream(p.meta + slab_off(rb, g, p.rb.meta) + lane * 16);
+  const uint32_t sc16 = ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * g, p.rb.scales));
   const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
   const uint32_t mw[4] = {mm.x, mm.y, mm.z, mm.w};
-  uint4* dst = reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + (uint64_t)g * 128);
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {             // 8 columns = 2 groups per 16-byte store
+  for (int c = 0; c < 16; ++c) {                     // 8 columns = 2 groups per 16-byte chunk
     uint32_t w[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int gi = 2 * c + h;
       const uint32_t pt = (mw[gi >> 3] >> (4 * (gi & 7))) & 15u;
+      const uint32_t i0 = (0x211000u >> (4 * pt)) & 15u, i1 = (0x332321u >> (4 * pt)) & 15u;
       const uint32_t byte = (vw[gi >> 2] >> (8 * (gi & 3))) & 0xFFu;
       const uint32_t q0 = int_to16((int)(byte & 15u) - 8, f16), q1 = int_to16((int)(byte >> 4) - 8, f16);
-      uint32_t lo = 0, hi = 0;               // columns (0,1) and (2,3) of the group
-      switch (pt) {
-        case 0: lo = q0 | (q1 << 16); break;                 // (0,1)
-        case 1: lo = q0; hi = q1; break;                     // (0,2)
-        case 2: lo = q0; hi = q1 << 16; break;               // (0,3)
-        case 3: lo = q0 << 16; hi = q1; break;               // (1,2)
-        case 4: lo = q0 << 16; hi = q1 << 16; break;         // (1,3)
-        default: hi = q0 | (q1 << 16); break;                // (2,3)
-      }
-      w[2 * h] = lo;
-      w[2 * h + 1] = hi;
+      w[2 * h] = (i0 == 0 ? q0 : 0u) | ((i0 == 1 ? q0 : (i1 == 1 ? q1 : 0u)) << 16);
+      w[2 * h + 1] = (i0 == 2 ? q0 : (i1 == 2 ? q1 : 0u)) | ((i1 == 3 ? q1 : 0u) << 16);
     }
-    dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    stage[warp][lane][c] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  scales[(uint64_t)n * G + g] = f16_bits_to_f32(ldg_u16(p.scales + rit(n, 2 * g, p.rb.scales)));
+  __syncwarp();
+  const int half = lane >> 4, c = lane & 15;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int row = 2 * i + half;
+    *reinterpret_cast<uint4*>(qbf + (uint64_t)(rb * 32 + row) * ldq + (uint64_t)g * 128 + c * 8) = stage[warp][row][c];
+  }
+  scales[(uint64_t)(rb * 32 + lane) * G + g] = f16_bits_to_f32(sc16);
 }
 
 // Any uniform codec with the 2:4 mask or no mask (generic bit extraction).
@@ -441,22 +445,29 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
 
 // Adapter columns of the main operand: [Lhi | Lhi | Llo | 0] at columns
 // K .. K + r3 of row n, with L^ = q_L s_L exact in fp32 and Lhi + Llo = L^.
+// A thread per (row, 8 columns): one 16-byte store.
 __global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3, int f16) {
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int r = p.d.rank;
-  if (id >= (uint64_t)p.d.n_out * r3) return;
-  const int n = (int)(id / r3), c = (int)(id % r3);
-  uint16_t v = 0;
-  if (c < 3 * r) {
-    const int j = c % r, part = c / r;                       // 0: hi, 1: hi, 2: lo
-    const uint32_t byte = p.l_values[rit(n, j / 2, p.rb.l_values)];
-    const int q = (int)((byte >> (4 * (j & 1))) & 15u) - 8;
-    const float s = f16_bits_to_f32(p.l_scales[(uint64_t)(n / kGroup) * r + j]);
-    const float l = (float)q * s;                            // exact (<= 14 significant bits)
-    const uint16_t hi = to16(l, f16);
-    v = part < 2 ? hi : to16(l - from16(hi, f16), f16);
+  const int r = p.d.rank, chunks = r3 / 8;
+  if (id >= (uint64_t)p.d.n_out * chunks) return;
+  const int n = (int)(id / chunks), c0 = (int)(id % chunks) * 8;
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = c0 + i;
+    uint32_t v = 0;
+    if (c < 3 * r) {
+      const int j = c % r, part = c / r;               // 0: hi, 1: hi, 2: lo
+      const uint32_t byte = p.l_values[rit(n, j / 2, p.rb.l_values)];
+      const int q = (int)((byte >> (4 * (j & 1))) & 15u) - 8;
+      const float sl = f16_bits_to_f32(p.l_scales[(uint64_t)(n / kGroup) * r + j]);
+      const float l = (float)q * sl;                     // exact (<= 14 significant bits)
+      const uint16_t hi = to16(l, f16);
+      v = part < 2 ? hi : to16(l - from16(hi, f16), f16);
+    }
+    w[i >> 1] |= v << (16 * (i & 1));
   }
-  qbf[(uint64_t)n * ldq + p.d.k_in + c] = v;
+  *reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + p.d.k_in + c0) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // R rows (padded to 128) as bf16 codes and fp32 scales.
@@ -589,12 +600,13 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   }
   const uint64_t nw = (uint64_t)N * G;
   if (p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM)
-    k_pf_dequant_w24<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc, f16);
+    k_pf_dequant_w24<<<(unsigned)(((uint64_t)p.n_rb * G + kDqWarps - 1) / kDqWarps), kDqWarps * 32, 0, st>>>(
+        p, qbf, L.ldq, wsc, f16);
   else
     k_pf_dequant_w<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc, f16);
   if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);       // main term off: zero scales
   if (lowrank) {
-    const uint64_t nl = (uint64_t)N * L.r3;
+    const uint64_t nl = (uint64_t)N * (L.r3 / 8);
     k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.r3, f16);
     const uint64_t nr = (uint64_t)L.rrows * K;
     k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows, f16);
