@@ -22,8 +22,9 @@
  * Conventions for every entry point
  *   - All data pointers are DEVICE pointers owned by the caller, except the
  *     descriptor/layout/output-scalar pointers, which are host pointers.
- *   - The library allocates no memory and keeps no global state.  Scratch
- *     memory comes from the caller's workspace.
+ *   - The library allocates no memory.  Scratch memory comes from the
+ *     caller's workspace (the one exception, compressed_linear_forward_noalloc,
+ *     uses a fixed scratch array inside the library instead).
  *   - Calls are stream-ordered and asynchronous.  Argument and format errors
  *     are returned synchronously before anything is launched.  Errors found
  *     on the device (a bad header, a bounded wait that ran out) are written to
@@ -218,12 +219,34 @@ cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t s
  *             batches run the tcgen05 tensor-core prefill GEMM, which is
  *             implemented for 2:4 int4 layers (others: CQL_ERR_UNSUPPORTED).
  *   workspace device, >= cql_workspace_size bytes, 256-byte aligned, zeroed
- *             once by cql_workspace_init.  Calls sharing one workspace must
- *             be ordered on one stream.
+ *             by cql_workspace_init before its first use with a given layer
+ *             and batch (the forward leaves it ready for the next call with
+ *             the same layer and batch).  Calls sharing one workspace must be
+ *             ordered on one stream.
  */
 cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, const void* x,
                                      cql_dtype x_dt, void* y, cql_dtype y_dt, int32_t batch,
                                      void* workspace, uint64_t ws_bytes, cql_stream_t stream);
+
+/* Forward pass without a workspace argument, for callers that cannot allocate
+ * device memory themselves: e.g. an inference-server plugin whose enqueue path
+ * may not allocate, a runtime that budgets every device byte ahead of time, or
+ * a binding that can only pass raw input and output pointers.  (This entry
+ * point is an addition of this library; the paper has no counterpart.)
+ *   Arguments as compressed_linear_forward, minus the workspace.  The scratch
+ *   memory is one fixed 4 MiB device array inside the library, held by every
+ *   GPU that loads it until the process exits; a call whose workspace
+ *   (cql_workspace_size) would exceed 4 MiB returns CQL_ERR_SIZE without
+ *   launching anything.  The library never calls cudaMalloc or cudaFree here.
+ *   The first call on a device finds the array's address and clears it (with
+ *   that device current; make this first call before any stream capture).
+ *   All calls share the array, and each call first clears (memset on its
+ *   stream) the part of it that it uses: calls that overlap on the GPU race,
+ *   so order them on one stream.  Device errors are recorded in the array's
+ *   error word and are not reported back by this entry point. */
+cql_status compressed_linear_forward_noalloc(const cql_desc* desc, const void* packed, const void* x,
+                                             cql_dtype x_dt, void* y, cql_dtype y_dt, int32_t batch,
+                                             cql_stream_t stream);
 
 /* Wait for the stream, then read and clear the device error word of a
  * workspace: *out = CQL_OK or the cql_status a kernel recorded. */

@@ -33,7 +33,7 @@ CQL_MAX_DECODE_BATCH = 16
 EXPORTED = (
     "cql_status_string", "cql_version", "cql_packed_layout", "cql_pack_workspace_size",
     "pack_compressed_weight", "cql_workspace_size", "cql_workspace_init",
-    "compressed_linear_forward", "cql_get_device_status",
+    "compressed_linear_forward", "cql_get_device_status", "compressed_linear_forward_noalloc",
 )
 
 
@@ -82,6 +82,8 @@ def lib():
         L.compressed_linear_forward.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P, ctypes.c_int,
                                                 I32, P, U64, P]
         L.cql_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+        L.compressed_linear_forward_noalloc.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P,
+                                                        ctypes.c_int, I32, P]
         for fn in EXPORTED[2:]:
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -163,6 +165,14 @@ def compressed_linear_forward(desc, packed, x, x_dt, y, y_dt, batch, workspace, 
     _check(lib().compressed_linear_forward(ctypes.byref(desc), _ptr(packed), _ptr(x), int(x_dt), _ptr(y), int(y_dt),
                                            int(batch), _ptr(workspace), int(ws_bytes), _stream(stream)),
            "compressed_linear_forward")
+
+
+def compressed_linear_forward_noalloc(desc, packed, x, x_dt, y, y_dt, batch, stream=None):
+    """Forward without a workspace (the library's fixed 4 MiB scratch array is
+    used instead); for callers that cannot allocate device memory."""
+    _check(lib().compressed_linear_forward_noalloc(ctypes.byref(desc), _ptr(packed), _ptr(x), int(x_dt), _ptr(y),
+                                                   int(y_dt), int(batch), _stream(stream)),
+           "compressed_linear_forward_noalloc")
 
 
 def cql_get_device_status(workspace, stream=None) -> int:
