@@ -35,13 +35,14 @@
 
 namespace cql {
 
-constexpr int kDecNT = 512;                    // threads per decode CTA (one CTA per SM)
-constexpr int kDecNW = kDecNT / 32;
-constexpr int kDepth = 4;                      // units in flight per warp (cp.async ring)
 constexpr int kDecSmem = 220 * 1024;           // shared memory per CTA: tables + ring
-template <int B> struct DecCfg {
-  static constexpr int kMinBlocks = 1;
-};
+
+// Offsets inside one plane fit in 32 bits (N * K <= 2^32 keeps every plane
+// below 4 GB), so the per-unit address arithmetic stays 32-bit.
+CQL_DEV uint32_t slab_off32(uint32_t rb, uint32_t s, uint32_t row_bytes) { return (rb * (row_bytes >> 4) + s) * 512u; }
+CQL_DEV uint32_t rit32(uint32_t i, uint32_t j, uint32_t row_bytes) {
+  return ((i >> 5) * (row_bytes >> 4) + (j >> 4)) * 512u + (i & 31u) * 16u + (j & 15u);
+}
 constexpr uint32_t kMagic = 0x4B000000u;       // fp32 bit pattern of 2^23
 
 CQL_DEV float act(const DecodeParams& p, int b, int col) {
@@ -97,6 +98,10 @@ CQL_DEV void pair_of(int pt, int& i0, int& i1) {
 
 template <int BITS, int B>
 struct Unit24 {
+  // batch 1 needs little register state: 32 warps per CTA, 2 units in flight
+  // each; larger batches keep more accumulators: 16 warps, 4 units in flight
+  static constexpr int kThreads = B == 1 ? 1024 : 512;
+  static constexpr int kDepth = B == 1 ? 2 : 4;
   static constexpr int NBP = B == 1 ? 1 : B / 2;                     // batch pairs
   static constexpr int kGroupBytes = B == 1 ? 64 : 128 * NBP;        // 8 patterns per group
   static constexpr int kTableBytes = 32 * kGroupBytes;
@@ -150,11 +155,11 @@ struct Unit24 {
   static constexpr int kSlabs = 3;
   static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
     const uint32_t vs = BITS == 4 ? 2u * uk : (24u * uk) >> 4;
-    const uint8_t* vb = p.values + slab_off(rb, vs, p.rb.values) + lane * 16;
+    const uint8_t* vb = p.values + slab_off32(rb, vs, p.rb.values) + lane * 16;
     cp_async16(slot, vb);
     cp_async16(slot + 512, vb + 512);
-    cp_async16(slot + 1024, p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
-    const uint32_t sc = ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    cp_async16(slot + 1024, p.meta + slab_off32(rb, uk, p.rb.meta) + lane * 16);
+    const uint32_t sc = ldg_u16(p.scales + rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales));
     return sc | (BITS == 3 && ((24u * uk) & 15u) ? 0x10000u : 0u);
   }
   static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
@@ -236,6 +241,8 @@ struct Unit24 {
 // ---------------------------------------------------------------------------
 template <int BITS, bool LUT, int B>
 struct UnitDense {
+  static constexpr int kThreads = 512;
+  static constexpr int kDepth = 4;
   static constexpr int kUnitBytes = kGroup * B * 4;        // x tile [128][B] fp32
   static constexpr int kWords = BITS * 4;                  // 128 codes = 16 or 12 words
   struct Frag {
@@ -261,10 +268,10 @@ struct UnitDense {
   }
   static constexpr int kSlabs = BITS;                     // 64 or 48 bytes of codes per unit
   static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
-    const uint8_t* vb = p.values + slab_off(rb, (uint64_t)BITS * uk, p.rb.values) + lane * 16;
+    const uint8_t* vb = p.values + slab_off32(rb, (uint32_t)BITS * uk, p.rb.values) + lane * 16;
 #pragma unroll
     for (int s = 0; s < BITS; ++s) cp_async16(slot + 512 * s, vb + 512 * s);
-    return LUT ? 0u : ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    return LUT ? 0u : ldg_u16(p.scales + rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales));
   }
   static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
 #pragma unroll
@@ -319,6 +326,8 @@ struct UnitDense {
 // ---------------------------------------------------------------------------
 template <int BITS, int B>
 struct UnitBitmap {
+  static constexpr int kThreads = 512;
+  static constexpr int kDepth = 4;
   static constexpr int kUnitBytes = kGroup * B * 4;        // x tile [128][B] fp32
   // 96-byte code window per lane: a unit's codes (<= 128 * BITS bits) start
   // at most 127 bits into the first slab, and the funnel shift also reads the
@@ -432,7 +441,9 @@ CQL_DEV bool header_ok(const DecodeParams& p) {
 }
 
 template <class U, int B>
-__global__ void __launch_bounds__(kDecNT, DecCfg<B>::kMinBlocks) k_decode(DecodeParams p, int ring_off) {
+__global__ void __launch_bounds__(U::kThreads, 1) k_decode(DecodeParams p, int ring_off) {
+  constexpr int kDepth = U::kDepth;
+  constexpr int kDecNW = U::kThreads / 32;
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_launch_dependents();                          // let the epilogue kernel get resident
@@ -700,7 +711,7 @@ static int sm_count() {
 
 template <class U, int B>
 static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, cudaStream_t st, bool pdl) {
-  const int ring = kDecNW * kDepth * U::kSlabs * 512;
+  const int ring = (U::kThreads / 32) * U::kDepth * U::kSlabs * 512;
   int ktu = (kDecSmem - ring - extra_bytes) / unit_bytes;
   ktu = max(1, min(ktu, p.upr));
   p.ktu = ktu;
@@ -717,11 +728,11 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  uint64_t grid = (uint64_t)sm_count() * DecCfg<B>::kMinBlocks;
+  uint64_t grid = (uint64_t)sm_count();
   if (grid > p.n_units) grid = p.n_units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kDecNT);
+  cfg.blockDim = dim3(U::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -755,11 +766,11 @@ static cudaError_t launch_main(const DecodeParams& p, cudaStream_t st, bool pdl)
     return launch_unit<Unit24<3, B>, B>(p, Unit24<3, B>::kUnitBytes, 0, st, pdl);
   }
   if (p.d.mask == CQL_MASK_BITMAP50) {
-    const int extra = kDecNW * UnitBitmap<4, B>::kWinWords * 32 * 4;
+    const int extra = (UnitBitmap<4, B>::kThreads / 32) * UnitBitmap<4, B>::kWinWords * 32 * 4;
     if (bits == 4) return launch_unit<UnitBitmap<4, B>, B>(p, UnitBitmap<4, B>::kUnitBytes, extra, st, pdl);
     return launch_unit<UnitBitmap<3, B>, B>(p, UnitBitmap<3, B>::kUnitBytes, extra, st, pdl);
   }
-  const int lut_extra = kDecNW * 16 * 32 * 4;
+  const int lut_extra = (UnitDense<3, true, B>::kThreads / 32) * 16 * 32 * 4;
   switch (p.d.codec) {
     case CQL_CODEC_INT4_SYM:
       return launch_unit<UnitDense<4, false, B>, B>(p, UnitDense<4, false, B>::kUnitBytes, 0, st, pdl);
