@@ -36,6 +36,7 @@
 namespace cql {
 
 constexpr int kDecSmem = 220 * 1024;           // shared memory per CTA: tables + ring
+constexpr int kEpiThreads = 64;                 // epilogue block: two row blocks (one row group)
 
 // Offsets inside one plane fit in 32 bits (N * K <= 2^32 keeps every plane
 // below 4 GB), so the per-unit address arithmetic stays 32-bit.
@@ -100,8 +101,8 @@ template <int BITS, int B>
 struct Unit24 {
   // batch 1 needs little register state: 32 warps per CTA, 2 units in flight
   // each; larger batches keep more accumulators: 16 warps, 4 units in flight
-  static constexpr int kThreads = B == 1 ? 1024 : 512;
-  static constexpr int kDepth = B == 1 ? 2 : 4;
+  static constexpr int kThreads = 512;
+  static constexpr int kDepth = 4;
   static constexpr int NBP = B == 1 ? 1 : B / 2;                     // batch pairs
   static constexpr int kGroupBytes = B == 1 ? 64 : 128 * NBP;        // 8 patterns per group
   static constexpr int kTableBytes = 32 * kGroupBytes;
@@ -534,59 +535,73 @@ __global__ void __launch_bounds__(U::kThreads, 1) k_decode(DecodeParams p, int r
 // accumulator and t only after.
 // ---------------------------------------------------------------------------
 template <int B>
-__global__ void __launch_bounds__(256, 1) k_epilogue(DecodeParams p, int kq) {
+__global__ void __launch_bounds__(kEpiThreads, 1) k_epilogue(DecodeParams p, int kq) {
+  // u[b][j] = s_L[g][j] * t[b][j] for this block's row group g (a block's
+  // kEpiThreads rows lie in one group of 128)
+  __shared__ float us[B * 256];
   const int lane = threadIdx.x & 31;
-  const int rb = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int rb = blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5);
   const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
-  if (rb >= p.n_rb) {
-    pdl_wait();
-    return;
-  }
+  const bool active = rb < p.n_rb;
   const int N = p.d.n_out, r = p.d.rank;
-  const int row = rb * 32 + lane, g = row / kGroup;
+  const int row = rb * 32 + lane;
+  const int g = (blockIdx.x * kEpiThreads) / kGroup;
   uint4 lv[8];
-  float ls[8];
 #pragma unroll
   for (int m = 0; m < 8; ++m) {                     // rank <= 256: at most 8 chunks of 32
     lv[m] = make_uint4(0u, 0u, 0u, 0u);
-    ls[m] = 0.0f;
-    if (lowrank && 32 * m < r) {
-      lv[m] = ldg_stream(p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
-      const int j = 32 * m + lane;
-      ls[m] = j < r ? f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) : 0.0f;
-    }
+    if (active && lowrank && 32 * m < r) lv[m] = ldg_stream(p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
   }
   pdl_wait();                                       // main term (and pre-kernel) complete
   float acc[B];
 #pragma unroll
   for (int b = 0; b < B; ++b) {
     acc[b] = 0.0f;
-    if (b < p.batch) {
-      float* a = p.y_acc + (uint64_t)b * N + row;
-      acc[b] = ld_cg_f32(a);
-      *a = 0.0f;
+    if (active && b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
+  }
+  if (lowrank) {
+    // every (b, j) of t: the K-slice partials, loaded four at a time
+    for (int i = threadIdx.x; i < B * r; i += kEpiThreads) {
+      const int b = i / r, j = i - b * r;
+      const float* tp = p.t_part + (uint64_t)b * p.r_pad + j;
+      const uint64_t st = (uint64_t)B * p.r_pad;
+      float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
+      int k = 0;
+      for (; k + 4 <= kq; k += 4) {
+        t0 += ld_cg_f32(tp + (k + 0) * st);
+        t1 += ld_cg_f32(tp + (k + 1) * st);
+        t2 += ld_cg_f32(tp + (k + 2) * st);
+        t3 += ld_cg_f32(tp + (k + 3) * st);
+      }
+      for (; k < kq; ++k) t0 += ld_cg_f32(tp + k * st);
+      us[i] = f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) * ((t0 + t1) + (t2 + t3));
     }
   }
+  __syncthreads();
+  if (!active) return;
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+    if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
   if (lowrank) {
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       if (32 * m >= r) break;
-      const int j = 32 * m + lane;
-      float u[B];
+      const uint32_t wd[4] = {lv[m].x, lv[m].y, lv[m].z, lv[m].w};
+      float q[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) q[jj] = (float)((int)((wd[jj >> 3] >> (4 * (jj & 7))) & 15u) - 8);
+      const int nj = min(32, r - 32 * m);           // 16 or 32
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        float t = 0.0f;
-        if (j < r)
-          for (int k = 0; k < kq; ++k) t += ld_cg_f32(p.t_part + ((uint64_t)k * B + b) * p.r_pad + j);
-        u[b] = ls[m] * t;
-      }
-      const uint32_t wd[4] = {lv[m].x, lv[m].y, lv[m].z, lv[m].w};
+        const float* ub = us + b * r + 32 * m;
+        float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        if (32 * m + jj >= r) break;
-        const float q = (float)((int)((wd[jj >> 3] >> (4 * (jj & 7))) & 15u) - 8);
+        for (int jj = 0; jj < 16; ++jj) a0 = fmaf(q[jj], ub[jj], a0);
+        if (nj == 32) {
 #pragma unroll
-        for (int b = 0; b < B; ++b) acc[b] = fmaf(q, __shfl_sync(0xffffffffu, u[b], jj), acc[b]);
+          for (int jj = 16; jj < 32; ++jj) a1 = fmaf(q[jj], ub[jj], a1);
+        }
+        acc[b] += a0 + a1;
       }
     }
   }
@@ -812,8 +827,8 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
   }
   int kq_arg = kq;
   void* args[2] = {&p, &kq_arg};
-  const dim3 grid((p.n_rb * 32 + 255) / 256);
-  return launch_pdl((const void*)k_epilogue<B>, args, grid, dim3(256), 0, st, main_on || p.has_pre);
+  const dim3 grid((p.n_rb * 32 + kEpiThreads - 1) / kEpiThreads);
+  return launch_pdl((const void*)k_epilogue<B>, args, grid, dim3(kEpiThreads), 0, st, main_on || p.has_pre);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st) {
