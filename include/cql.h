@@ -62,9 +62,11 @@
  *         lut3/lut4: index of the row's centroid.
  *         kept per row = K/2 under 2:4 and bitmap50, K without a mask.
  *         row_bytes = pad16(ceil(kept * b / 8)).
- * META    2:4: 4-bit pattern index p of column group g (columns 4g..4g+3) at
- *         stream bits [4g, 4g+4); p names the kept pair (i0, i1), i0 < i1, in
- *         lexicographic order: 0:(0,1) 1:(0,2) 2:(0,3) 3:(1,2) 4:(1,3) 5:(2,3).
+ * META    2:4: 4-bit code of column group g (columns 4g..4g+3) at stream
+ *         bits [4g, 4g+4): the kept positions themselves, i0 | (i1 << 2),
+ *         i0 < i1 (the 2-bit-index form sparse tensor cores read; valid codes
+ *         0x4 0x8 0xC 0x9 0xD 0xE).  The kept codes of the group are, in
+ *         VALUES, those of columns 4g+i0 then 4g+i1.
  *         bitmap50: bit k of the row stream is 1 when column k is kept.
  *         row_bytes = K/8.  Absent without a mask.
  * SCALES  int4/int3: fp16 scale of columns [128g, 128g+128) at row bytes

@@ -42,7 +42,7 @@ import numpy as np
 __all__ = [
     "MASK_NONE", "MASK_2_4", "MASK_BITMAP50",
     "CODEC_INT4", "CODEC_INT3", "CODEC_LUT3", "CODEC_LUT4",
-    "GROUP", "ROWBLK", "PAIRS_2OF4",
+    "GROUP", "ROWBLK", "PAIRS_2OF4", "META_NIBBLE_2OF4",
     "OracleDesc", "desc_for",
     "fp16_round", "n_outliers", "select_outliers",
     "mask_2of4", "mask_bitmap50",
@@ -66,6 +66,10 @@ SLAB = 16              # bytes each row contributes to one slab
 
 # 2:4 pattern index p -> kept positions (i0, i1), i0 < i1, lexicographic.
 PAIRS_2OF4 = ((0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3))
+# Byte-format code of a 2:4 group in the META plane: the two kept positions
+# themselves, i0 | (i1 << 2) (a format choice: the pages fix no byte layout;
+# this is the 2-bit-index form that sparse tensor cores read).
+META_NIBBLE_2OF4 = tuple(i0 | (i1 << 2) for i0, i1 in PAIRS_2OF4)
 
 _CODEC_BITS = {CODEC_INT4: 4, CODEC_INT3: 3, CODEC_LUT3: 3, CODEC_LUT4: 4}
 
@@ -593,7 +597,8 @@ def pack_bytes(desc: OracleDesc, parts: Dict[str, np.ndarray]) -> np.ndarray:
         kept_codes = codes[keep].reshape(n, kept)   # row-major boolean index keeps column order
     put(P_VALUES, _interleave(_bitstream(kept_codes, bits, rb[P_VALUES])))
     if desc.mask == MASK_2_4:
-        put(P_META, _interleave(_bitstream(parts["pattern"], 4, rb[P_META])))
+        nib = np.asarray(META_NIBBLE_2OF4, dtype=np.uint8)[parts["pattern"]]
+        put(P_META, _interleave(_bitstream(nib, 4, rb[P_META])))
     elif desc.mask == MASK_BITMAP50:
         put(P_META, _interleave(_bitstream(keep.astype(np.uint8), 1, rb[P_META])))
     if desc.codec in (CODEC_INT4, CODEC_INT3):

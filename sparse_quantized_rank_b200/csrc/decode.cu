@@ -10,9 +10,10 @@
 //  * Because all lanes of a warp sit on the same columns, the activations are
 //    warp-uniform.  For the 2:4 mask the x pair a kept pair multiplies,
 //    (x[4g+i0], x[4g+i1]), is read from a shared-memory table indexed by the
-//    group and the pattern nibble (6 patterns): at most 6 distinct addresses
-//    per warp access, all in distinct banks, so one wavefront.  The metadata
-//    nibble becomes a table offset with a shift and a mask.
+//    group and the META code (the kept positions, i0 | i1 << 2; 6 valid
+//    codes): at most 6 distinct addresses per warp access, all in distinct
+//    banks, so one wavefront.  The code becomes a table offset with a shift
+//    and a mask.
 //  * int4 codes are turned into floats two at a time with byte permutes into
 //    the 2^23 magic exponent and one packed fp32x2 subtraction; the products
 //    are packed fp32x2 FMAs.  The group scale multiplies the group's partial
@@ -104,7 +105,7 @@ struct Unit24 {
   static constexpr int kThreads = 512;
   static constexpr int kDepth = 4;
   static constexpr int NBP = B == 1 ? 1 : B / 2;                     // batch pairs
-  static constexpr int kGroupBytes = B == 1 ? 64 : 128 * NBP;        // 8 patterns per group
+  static constexpr int kGroupBytes = B == 1 ? 128 : 256 * NBP;       // 16 entries per group (by META code)
   static constexpr int kTableBytes = 32 * kGroupBytes;
   static constexpr int kUnitBytes = kTableBytes + kGroup * B * 4;   // table + staged x
   struct Frag {
@@ -113,8 +114,9 @@ struct Unit24 {
     uint32_t s;
   };
 
-  // Pair table of the K tile: entry (group, pattern) = the x values of the
-  // pattern's two kept columns (B == 1), or of two batches (B >= 2).
+  // Pair table of the K tile: entry (group, META code i0 | i1 << 2) = the x
+  // values of columns i0 and i1 (B == 1), or of two batches (B >= 2); only
+  // the six valid codes are written.
   static CQL_DEV void build(const DecodeParams& p, uint8_t* smem, int kt) {
     const int c0 = kt * p.ktu * kGroup;
     const int units = min(p.ktu, p.upr - kt * p.ktu);
@@ -129,22 +131,23 @@ struct Unit24 {
       const float* xc = xs + (4 * g) * B + 2 * bp;
       if (B == 1) {
         const float4 x4 = *reinterpret_cast<const float4*>(xc);
-        float4* e = reinterpret_cast<float4*>(smem + g * 64);
-        e[0] = make_float4(x4.x, x4.y, x4.x, x4.z);   // patterns 0 (0,1), 1 (0,2)
-        e[1] = make_float4(x4.x, x4.w, x4.y, x4.z);   // patterns 2 (0,3), 3 (1,2)
-        e[2] = make_float4(x4.y, x4.w, x4.z, x4.w);   // patterns 4 (1,3), 5 (2,3)
+        uint8_t* e = smem + g * 128;                   // 8 bytes per code
+        *reinterpret_cast<float2*>(e + 8 * 0x4) = make_float2(x4.x, x4.y);                 // (0,1)
+        *reinterpret_cast<float4*>(e + 8 * 0x8) = make_float4(x4.x, x4.z, x4.y, x4.z);     // (0,2) (1,2)
+        *reinterpret_cast<float4*>(e + 8 * 0xC) = make_float4(x4.x, x4.w, x4.y, x4.w);     // (0,3) (1,3)
+        *reinterpret_cast<float2*>(e + 8 * 0xE) = make_float2(x4.z, x4.w);                 // (2,3)
       } else {
         const float2 c0v = *reinterpret_cast<const float2*>(xc);          // column 0, batches b, b+1
         const float2 c1v = *reinterpret_cast<const float2*>(xc + B);
         const float2 c2v = *reinterpret_cast<const float2*>(xc + 2 * B);
         const float2 c3v = *reinterpret_cast<const float2*>(xc + 3 * B);
-        float4* e = reinterpret_cast<float4*>(smem + (g * NBP + bp) * 128);
-        e[0] = make_float4(c0v.x, c1v.x, c0v.y, c1v.y);
-        e[1] = make_float4(c0v.x, c2v.x, c0v.y, c2v.y);
-        e[2] = make_float4(c0v.x, c3v.x, c0v.y, c3v.y);
-        e[3] = make_float4(c1v.x, c2v.x, c1v.y, c2v.y);
-        e[4] = make_float4(c1v.x, c3v.x, c1v.y, c3v.y);
-        e[5] = make_float4(c2v.x, c3v.x, c2v.y, c3v.y);
+        float4* e = reinterpret_cast<float4*>(smem + (g * NBP + bp) * 256);   // 16 bytes per code
+        e[0x4] = make_float4(c0v.x, c1v.x, c0v.y, c1v.y);
+        e[0x8] = make_float4(c0v.x, c2v.x, c0v.y, c2v.y);
+        e[0xC] = make_float4(c0v.x, c3v.x, c0v.y, c3v.y);
+        e[0x9] = make_float4(c1v.x, c2v.x, c1v.y, c2v.y);
+        e[0xD] = make_float4(c1v.x, c3v.x, c1v.y, c3v.y);
+        e[0xE] = make_float4(c2v.x, c3v.x, c2v.y, c3v.y);
       }
     }
   }
@@ -200,14 +203,14 @@ struct Unit24 {
     const uint32_t mw = f.m[GI >> 3];
     constexpr int jn = GI & 7;
     if (B == 1) {
-      const uint32_t off = jn == 0 ? ((mw << 3) & 0x38u) : ((mw >> (4 * jn - 3)) & 0x38u);
-      const uint64_t xp = *reinterpret_cast<const uint64_t*>(tb + GI * 64 + off);
+      const uint32_t off = jn == 0 ? ((mw << 3) & 0x78u) : ((mw >> (4 * jn - 3)) & 0x78u);
+      const uint64_t xp = *reinterpret_cast<const uint64_t*>(tb + GI * 128 + off);
       a2[0] = f2_fma(qq, xp, a2[0]);
     } else {
-      const uint32_t off = jn == 0 ? ((mw << 4) & 0x70u) : ((mw >> (4 * jn - 4)) & 0x70u);
+      const uint32_t off = jn == 0 ? ((mw << 4) & 0xF0u) : ((mw >> (4 * jn - 4)) & 0xF0u);
 #pragma unroll
       for (int bp = 0; bp < NBP; ++bp) {
-        const ulonglong2 e = *reinterpret_cast<const ulonglong2*>(tb + (GI * NBP + bp) * 128 + off);
+        const ulonglong2 e = *reinterpret_cast<const ulonglong2*>(tb + (GI * NBP + bp) * 256 + off);
         a2[2 * bp] = f2_fma(qq, e.x, a2[2 * bp]);
         a2[2 * bp + 1] = f2_fma(qq, e.y, a2[2 * bp + 1]);
       }

@@ -287,14 +287,9 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
       }
       keep = rank < 2;
       const uint32_t m4 = (__ballot_sync(0xffffffffu, keep) >> q0) & 15u;
-      switch (m4) {
-        case 0x3: pat = 0; break;
-        case 0x5: pat = 1; break;
-        case 0x9: pat = 2; break;
-        case 0x6: pat = 3; break;
-        case 0xA: pat = 4; break;
-        default: pat = 5; break;      // 0xC
-      }
+      // kept positions i0 < i1 of the group -> META code i0 | (i1 << 2)
+      const int i0 = __ffs(m4) - 1, i1 = 31 - __clz(m4);
+      pat = i0 | (i1 << 2);
     } else if (MASK == CQL_MASK_BITMAP50) {
       keep = (p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u;
     }

@@ -345,7 +345,8 @@ CQL_DEV uint16_t int_to16(int q, int f16) { return to16((float)q, f16); }   // e
 
 // 2:4 int4 -> 16-bit codes, zeros where pruned.  A warp per (row block,
 // 128-column unit): coalesced 16-byte loads of its code and pattern slabs
-// (lane = row), branch-free expansion of each group, a transpose through
+// (lane = row), branch-free expansion of each group (its META code holds the
+// kept positions i0 | i1 << 2), a transpose through
 // shared memory, then full-row 16-byte stores (two rows per instruction).
 constexpr int kDqWarps = 4;
 __global__ void __launch_bounds__(kDqWarps * 32) k_pf_dequant_w24(DecodeParams p, uint16_t* qbf, int ldq,
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(kDqWarps * 32) k_pf_dequant_w24(DecodeParams p
     for (int h = 0; h < 2; ++h) {
       const int gi = 2 * c + h;
       const uint32_t pt = (mw[gi >> 3] >> (4 * (gi & 7))) & 15u;
-      const uint32_t i0 = (0x211000u >> (4 * pt)) & 15u, i1 = (0x332321u >> (4 * pt)) & 15u;
+      const uint32_t i0 = pt & 3u, i1 = pt >> 2;
       const uint32_t byte = (vw[gi >> 2] >> (8 * (gi & 3))) & 0xFFu;
       const uint32_t q0 = int_to16((int)(byte & 15u) - 8, f16), q1 = int_to16((int)(byte >> 4) - 8, f16);
       w[2 * h] = (i0 == 0 ? q0 : 0u) | ((i0 == 1 ? q0 : (i1 == 1 ? q1 : 0u)) << 16);
@@ -403,8 +404,7 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
     for (int gi = 0; gi < 32; ++gi) {
       const uint32_t mb = p.meta[rit(n, (uint64_t)g * 16 + gi / 2, p.rb.meta)];
       const uint32_t pt = (mb >> (4 * (gi & 1))) & 15u;
-      const int i0 = pt < 3 ? 0 : (pt < 5 ? 1 : 2);
-      const int i1 = pt == 0 ? 1 : (pt == 1 || pt == 3 ? 2 : 3);
+      const int i0 = (int)(pt & 3u), i1 = (int)(pt >> 2);
       int qv[2];
       for (int h = 0; h < 2; ++h) {
         const uint64_t bp = bit0 + (uint64_t)bits * (2 * gi + h);

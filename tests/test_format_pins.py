@@ -94,8 +94,8 @@ def test_packed_bytes_decode_to_parts(name, over):
         if d.mask == O.MASK_2_4:
             meta = plane(O.P_META)
             for g in range(k // 4):
-                p = read_bits(meta, i, k // 8, 4 * g, 4)
-                i0, i1 = O.PAIRS_2OF4[p]
+                nib = read_bits(meta, i, k // 8, 4 * g, 4)
+                i0, i1 = nib & 3, nib >> 2
                 assert [c - 4 * g for c in cols if 4 * g <= c < 4 * g + 4] == [i0, i1]
         elif d.mask == O.MASK_BITMAP50:
             meta = plane(O.P_META)
