@@ -31,6 +31,12 @@ CQL_HD uint64_t rit(uint64_t i, uint64_t j, uint64_t row_bytes) {
 CQL_HD uint64_t slab_off(uint64_t rb, uint64_t s, uint64_t row_bytes) {
   return (rb * (row_bytes >> 4) + s) * 512u;
 }
+// Offsets inside one plane fit in 32 bits (N * K <= 2^32 keeps every plane
+// below 4 GB), so the per-unit address arithmetic stays 32-bit.
+CQL_DEV uint32_t slab_off32(uint32_t rb, uint32_t s, uint32_t row_bytes) { return (rb * (row_bytes >> 4) + s) * 512u; }
+CQL_DEV uint32_t rit32(uint32_t i, uint32_t j, uint32_t row_bytes) {
+  return ((i >> 5) * (row_bytes >> 4) + (j >> 4)) * 512u + (i & 31u) * 16u + (j & 15u);
+}
 
 // Per-plane row bytes of the packed format (see include/cql.h).
 struct RowBytes {
@@ -155,6 +161,16 @@ CQL_DEV float ld_cg_f32(const float* p) {
 }
 
 // Programmatic dependent launch controls (no-ops without a PDL edge).
+// 16-byte asynchronous global -> shared copies (LSU path), grouped per thread.
+CQL_DEV void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+CQL_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+CQL_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 CQL_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 CQL_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

@@ -39,26 +39,12 @@ namespace cql {
 constexpr int kDecSmem = 220 * 1024;           // shared memory per CTA: tables + ring
 constexpr int kEpiThreads = 64;                 // epilogue block: two row blocks (one row group)
 
-// Offsets inside one plane fit in 32 bits (N * K <= 2^32 keeps every plane
-// below 4 GB), so the per-unit address arithmetic stays 32-bit.
-CQL_DEV uint32_t slab_off32(uint32_t rb, uint32_t s, uint32_t row_bytes) { return (rb * (row_bytes >> 4) + s) * 512u; }
-CQL_DEV uint32_t rit32(uint32_t i, uint32_t j, uint32_t row_bytes) {
-  return ((i >> 5) * (row_bytes >> 4) + (j >> 4)) * 512u + (i & 31u) * 16u + (j & 15u);
-}
 constexpr uint32_t kMagic = 0x4B000000u;       // fp32 bit pattern of 2^23
 
 CQL_DEV float act(const DecodeParams& p, int b, int col) {
   return b < p.batch ? to_f32_act(p.x, p.xdt, (uint64_t)b * p.d.k_in + col) : 0.0f;
 }
 
-CQL_DEV void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
-               "l"(gsrc)
-               : "memory");
-}
-CQL_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-CQL_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 CQL_DEV uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
 // Activations x[b][c0, c0 + ncols) -> fp32 xs[c * B + b] in shared memory,
@@ -437,12 +423,6 @@ CQL_DEV void unit_coords(const DecodeParams& p, uint64_t u, int& kt, int& rb, in
   ut = (int)(r % s);
 }
 
-CQL_DEV bool header_ok(const DecodeParams& p) {
-  const uint32_t* h = reinterpret_cast<const uint32_t*>(p.header);
-  const int32_t* d = reinterpret_cast<const int32_t*>(p.header + 8);
-  return h[0] == 0x314C5143u /* "CQL1" */ && h[1] == CQL_VERSION && d[0] == p.d.n_out && d[1] == p.d.k_in &&
-         d[2] == p.d.mask && d[3] == p.d.codec && d[7] == p.d.rank;
-}
 
 template <class U, int B>
 __global__ void __launch_bounds__(U::kThreads, 1) k_decode(DecodeParams p, int ring_off) {
@@ -714,7 +694,7 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
 // ---------------------------------------------------------------------------
 // host launch
 // ---------------------------------------------------------------------------
-static int sm_count() {
+int device_sm_count() {
   static int cache[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -746,7 +726,7 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  uint64_t grid = (uint64_t)sm_count();
+  uint64_t grid = (uint64_t)device_sm_count();
   if (grid > p.n_units) grid = p.n_units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -826,7 +806,8 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
   }
   const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
   if (main_on) {
-    if ((e = launch_main<B>(p, st, p.has_pre)) != cudaSuccess) return e;
+    e = decode_tc_eligible(p) ? launch_decode_tc(p, B, st, p.has_pre) : launch_main<B>(p, st, p.has_pre);
+    if (e != cudaSuccess) return e;
   }
   int kq_arg = kq;
   void* args[2] = {&p, &kq_arg};

@@ -1,0 +1,445 @@
+// Decode main term on the sparse tensor cores: 2:4 mask, int4 codes, batch
+// 1..16.  y_acc[b][n] += sum_g s[n][g] * sum_{k in g} q[n][k] x[b][k]
+// (SLiM-Quant's per-group scale on a 2:4-pruned matrix, SLiM review summary
+// "SLIM-Quant"; the 2:4 pattern is what the sparse tensor cores execute).
+//
+// A tile is 128 weight rows x one scale group (128 columns).  Per tile:
+//   * each converter warp fetches its 32-row block's packed bytes (two code
+//     slabs and one META slab, 16 bytes per lane each) with cp.async, several
+//     tiles ahead; x (the MMA's B operand, batch padded to 16 rows with zeros)
+//     arrives in chunks of 1024 columns, one 3-D TMA box per chunk;
+//   * a converter warpgroup (lanes = rows, as the planes are laid out) turns
+//     the 64 kept codes of each row into exact bf16/f16 integers and writes
+//     them straight into tensor memory (compressed A, 32 columns), and writes
+//     the META codes, regrouped across lanes into the order the sparse MMA
+//     reads them, next to it;
+//   * the MMA warp issues four tcgen05.mma.sp (M 128, N 16, K 32) into a
+//     fresh fp32 accumulator in tensor memory;
+//   * the converter warpgroup reads the accumulator back (lane = row), scales
+//     it by the row's fp32 group scale and sums over the tile's row tile;
+//     partial row sums go to y_acc with reductions at L2 (split-K across
+//     CTAs), where the epilogue kernel adds the adapter term and rounds.
+// The scale is applied outside the MMA so that no dequantised weight is ever
+// rounded to 16 bits: the tensor cores multiply exact integers.
+//
+// Roles (640 threads, one CTA per SM, persistent over a contiguous tile range):
+//   warps 0..3    MMA issuer of converter warpgroup 0..3 (one lane each);
+//                 warp 0 also allocates tensor memory and loads the x chunks
+//   warps 4..19   converter warpgroups 0..3 (tile k of the range goes to
+//                 warpgroup k mod 4); each warp fetches its own row block's
+//                 packed bytes with cp.async into a private ring
+// Every mbarrier wait is bounded; on expiry the kernel records
+// CQL_ERR_TIMEOUT and winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace cql {
+namespace {
+
+constexpr int TC_WG = 4;                          // converter warpgroups
+constexpr int TC_THREADS = 128 * (1 + TC_WG);     // warps 0..3 MMA issuers, then the warpgroups
+constexpr int TC_KC = 8;                          // scale groups per x chunk (1024 columns)
+constexpr int TC_RING = 4;                        // tiles in flight per converter warp (cp.async ring)
+constexpr int TC_TS = 2;                          // tensor-memory stages per converter warpgroup
+constexpr int TC_VAL_BYTES = 1024;                // codes of one 32-row block: 2 slabs
+constexpr int TC_META_BYTES = 512;                // META of one 32-row block: 1 slab
+constexpr int TC_SLOT_BYTES = TC_VAL_BYTES + TC_META_BYTES + 512;   // one row block of one tile (+ scale slab)
+constexpr int TC_XBOX_BYTES = 16 * 64 * 2;        // TMA box: 16 rows x 64 columns of 16-bit x
+constexpr int TC_XCHUNK_BYTES = TC_KC * 2 * TC_XBOX_BYTES;
+
+// Tensor-memory columns of converter warpgroup w (512 allocated, 128 each):
+//   A (compressed codes) stage s: 128 w + 32 s          (32 columns)
+//   D (fp32 accumulator) stage s: 128 w + 64 + 16 s     (16 columns)
+//   META stage s:                 128 w + 96 + 8 s      (8 columns: K steps 0, 1 at
+//                                 +0, +1 and 2, 3 at +4, +5)
+// The sparse MMA takes its metadata address aligned and the column inside the
+// aligned pair from the instruction descriptor's selector bits [0, 2).
+CQL_HD uint32_t col_a(int w, int s) { return 128u * w + 32u * s; }
+CQL_HD uint32_t col_d(int w, int s) { return 128u * w + 64u + 16u * s; }
+CQL_HD uint32_t col_m(int w, int s) { return 128u * w + 96u + 8u * s; }
+
+struct TcSmem {
+  uint8_t x[2][TC_XCHUNK_BYTES];                  // x chunks, 1024-byte aligned (128-byte swizzle atoms)
+  uint8_t bias[128 * 128];                        // constant A of the offset MMA (all elements equal)
+  uint8_t ring[4 * TC_WG][TC_RING][TC_SLOT_BYTES];   // per converter warp: [values 1024][META 512][scales 512]
+  int slot_rt[4 * TC_WG][TC_RING];                // row tile and group of each ring slot
+  int slot_g[4 * TC_WG][TC_RING];
+  float scale[TC_WG][TC_TS][128];                 // group scale of each row of a tensor-memory stage
+  int tinfo[TC_WG][TC_TS][4];                     // row tile of a stage (one copy per converter warp)
+  uint64_t afull[TC_WG][TC_TS], dfull[TC_WG][TC_TS];
+  uint64_t xfull[2], xempty[2];
+  uint32_t tmem_base;
+};
+
+struct TcGeom {
+  int n_rt;          // row tiles (N / 128)
+  int G;             // scale groups per row (K / 128)
+  int n_chunks;      // ceil(G / TC_KC)
+  int n_tiles;       // n_rt * G  (N K <= 2^32 keeps it below 2^18)
+};
+
+// Tile order: x chunk, then row tile, then group inside the chunk, so that a
+// CTA's contiguous range touches one or two x chunks and runs along K inside
+// a row tile.
+CQL_DEV void tile_coords(const TcGeom& g, int t, int& c, int& rt, int& grp) {
+  const int per_full = g.n_rt * TC_KC;
+  const int cc = min(t / per_full, g.n_chunks - 1);
+  const int r = t - cc * per_full;
+  const int gc = min(TC_KC, g.G - cc * TC_KC);
+  c = cc;
+  rt = r / gc;
+  grp = cc * TC_KC + (r - rt * gc);
+}
+
+// Walks the tile order without divisions: (chunk, row tile, group in chunk).
+struct TileIter {
+  int c, rt, gl, gc, g;
+  CQL_DEV void init(const TcGeom& geo, int t) {
+    if (t >= geo.n_tiles) t = geo.n_tiles - 1;      // past the end: any valid tile (never used)
+    tile_coords(geo, t, c, rt, g);
+    gc = min(TC_KC, geo.G - c * TC_KC);
+    gl = g - c * TC_KC;
+  }
+  // advance by 'steps' tiles (steps <= one chunk's tiles)
+  CQL_DEV void advance(const TcGeom& geo, int steps) {
+    gl += steps;
+    while (gl >= gc) {
+      gl -= gc;
+      if (++rt == geo.n_rt) {
+        rt = 0;
+        if (c + 1 < geo.n_chunks) ++c;
+        gc = min(TC_KC, geo.G - c * TC_KC);
+      }
+    }
+    g = c * TC_KC + gl;
+  }
+  CQL_DEV void next(const TcGeom& geo) {
+    if (++gl == gc) {
+      gl = 0;
+      if (++rt == geo.n_rt) {
+        rt = 0;
+        if (c + 1 < geo.n_chunks) ++c;
+        gc = min(TC_KC, geo.G - c * TC_KC);
+      }
+    }
+    g = c * TC_KC + gl;
+  }
+};
+
+// One 2:4 group's two codes u as exact 16-bit floats u + 128 (bf16) or
+// u + 1024 (f16).  'lo' holds the group's byte (low nibble: code of the first
+// kept column), 'hi' the same word shifted right by 4.  The byte permute puts
+// the two nibbles at bits 0 and 16; the LOP3 masks them and ORs in the
+// exponent of 128 (bf16: 0x4300) or 1024 (f16: 0x6400).  The offset, with the
+// code bias 8 (q = u - 8), is removed by a second MMA over the same kept
+// positions with a constant A of -136 (bf16) or -1032 (f16), so
+//   D = sum (u + 128) x - 136 sum x = sum q x     (bf16; f16 alike),
+// exact products in fp32 accumulation.
+template <bool F16>
+CQL_DEV uint32_t code_pair(uint32_t lo, uint32_t hi, uint32_t sel) {
+  const uint32_t t = prmt(lo, hi, sel);
+  uint32_t a;
+  constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(t), "r"(0x000F000Fu), "r"(magic));
+  return a;
+}
+constexpr uint32_t kBiasBf16x2 = 0xC308C308u;     // -136, -136
+constexpr uint32_t kBiasF16x2 = 0xE408E408u;      // -1032, -1032
+
+// Instruction descriptor: sparse, D f32, A = B = bf16 (or f16), K-major,
+// M = 128, N = 16.
+CQL_HD uint32_t tc_idesc(bool f16) {
+  const uint32_t fmt = f16 ? 0u : 1u;
+  return (1u << 2) | (1u << 4) | (fmt << 7) | (fmt << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+template <int B, bool F16>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_decode_tc(const __grid_constant__ CUtensorMap tmX, DecodeParams p, TcGeom geo) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();                          // let the epilogue kernel get resident
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
+
+  const int t0 = (int)((uint64_t)geo.n_tiles * blockIdx.x / gridDim.x);
+  const int t1 = (int)((uint64_t)geo.n_tiles * (blockIdx.x + 1) / gridDim.x);
+  const int n = t1 - t0;
+
+  {
+    const uint32_t bv = F16 ? kBiasF16x2 : kBiasBf16x2;
+    for (int i = threadIdx.x; i < 128 * 128 / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(S.bias)[i] = make_uint4(bv, bv, bv, bv);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+  }
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < TC_WG; ++w)
+      for (int s = 0; s < TC_TS; ++s) {
+        mbar_init(&S.afull[w][s], 4);
+        mbar_init(&S.dfull[w][s], 1);
+      }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.xfull[b], 1);
+      mbar_init(&S.xempty[b], TC_WG);               // one commit from each MMA issuer
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&S.tmem_base))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp < TC_WG) {
+    // ---------------- MMA issuer of warpgroup w (one lane) ----------------
+    // A thread pays ~120 cycles per tcgen05.mma it issues; issuers in
+    // different warps overlap, so each warpgroup has its own.  Issuer 0 also
+    // loads the x chunks (one 3-D TMA box each), one chunk ahead.  x chunk c
+    // uses buffer c & 1; the chunks of the range are consecutive, so the
+    // phase of a buffer follows from the chunk index.
+    if (lane == 0 && n > 0) {
+      const int w = warp;
+      bool ok = true;
+      TileIter first, last;
+      first.init(geo, t0);
+      last.init(geo, t1 - 1);
+      const int c0 = first.c, c1 = last.c;
+      auto phase = [&](int c) { return (uint32_t)(((c - c0) >> 1) & 1); };   // use index of buffer c & 1
+      if (w == 0) {
+        for (int c = c0; c <= min(c0 + 1, c1); ++c) {
+          mbar_expect_tx(&S.xfull[c & 1], TC_XCHUNK_BYTES);
+          tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
+        }
+      }
+      int cur_c = -1, xc = -1;                      // chunk retired up to / chunk whose x is acquired
+      uint32_t xb = 0;
+      const uint32_t idesc = tc_idesc(F16);
+      const uint64_t dbias = smem_desc_sw128(smem_u32(S.bias));
+      TileIter it;
+      it.init(geo, t0 + w);
+      for (int k = w; ok; k += TC_WG, it.advance(geo, TC_WG)) {
+        const int c = k < n ? it.c : c1 + 1;        // past the end: retire every remaining chunk
+        for (; cur_c < c && ok;) {
+          if (cur_c >= 0) {
+            tc_commit(&S.xempty[cur_c & 1]);        // free once this issuer's MMAs on it finish
+            if (w == 0 && cur_c + 2 <= c1) {        // chunk cur_c + 2 reuses that buffer
+              const int cn = cur_c + 2, b = cn & 1;
+              if (!mbar_wait(&S.xempty[b], phase(cn) ^ 1)) { ok = false; break; }
+              mbar_expect_tx(&S.xfull[b], TC_XCHUNK_BYTES);
+              tma_load_3d(S.x[b], &tmX, &S.xfull[b], 0, 0, cn * 2 * TC_KC);
+            }
+          }
+          cur_c = cur_c < 0 ? c0 : cur_c + 1;
+        }
+        if (!ok || k >= n) break;
+        if (c != xc) {
+          const int b = c & 1;
+          if (!mbar_wait(&S.xfull[b], phase(c))) { ok = false; break; }
+          xb = smem_u32(S.x[b]);
+          xc = c;
+          tc_fence_after();
+        }
+        const int i = k / TC_WG, ts = i % TC_TS;
+        if (!mbar_wait(&S.afull[w][ts], (i / TC_TS) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t xg = xb + (uint32_t)(2 * it.gl) * TC_XBOX_BYTES;
+        const uint32_t d = tmem + col_d(w, ts), a = tmem + col_a(w, ts), m = tmem + col_m(w, ts);
+        const uint64_t b0 = smem_desc_sw128(xg), b1 = smem_desc_sw128(xg + 64);
+        const uint64_t b2 = smem_desc_sw128(xg + TC_XBOX_BYTES), b3 = smem_desc_sw128(xg + TC_XBOX_BYTES + 64);
+        tc_mma_sp_ta(d, a, b0, m, idesc, 0u);
+        tc_mma_sp_ta(d, a + 8, b1, m, idesc | 1u, 1u);
+        tc_mma_sp_ta(d, a + 16, b2, m + 4, idesc, 1u);
+        tc_mma_sp_ta(d, a + 24, b3, m + 4, idesc | 1u, 1u);
+        tc_mma_sp_ss(d, dbias, b0, m, idesc, 1u);
+        tc_mma_sp_ss(d, dbias, b1, m, idesc | 1u, 1u);
+        tc_mma_sp_ss(d, dbias, b2, m + 4, idesc, 1u);
+        tc_mma_sp_ss(d, dbias, b3, m + 4, idesc | 1u, 1u);
+        tc_commit(&S.dfull[w][ts]);
+      }
+      if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 21);
+    }
+  } else {
+    // ---------------- converter / accumulator warpgroups ----------------
+    const int w = (warp >> 2) - 1, qq = warp & 3;   // qq: tensor-memory lane quarter = row block of the tile
+    const int cw = warp - 4;                        // converter warp index
+    const int nw = (n - w + TC_WG - 1) / TC_WG;     // tiles of this warpgroup: k = TC_WG i + w
+    const uint32_t lane_base = (uint32_t)(32 * qq) << 16;
+    const uint32_t sel_meta = (lane & 8) ? 0x3276u : 0x5410u;
+    const uint32_t srow = 32u * qq + lane;          // row inside the tile
+    float acc[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+    bool ok = true;
+    // This warp's ring: lane l copies, and later reads back, only its own row's
+    // 16-byte pieces (codes, META, the scale slab piece holding its group's
+    // scale), so no cross-lane synchronisation is needed for them.
+    uint8_t* ring = S.ring[cw][0] + lane * 16;
+    const uint32_t vstride = (p.rb.values >> 4) * 512u, mstride = (p.rb.meta >> 4) * 512u;
+    const uint32_t sstride = (p.rb.scales >> 4) * 512u;
+    TileIter ld;                                    // next tile to fetch
+    ld.init(geo, t0 + w);
+    auto fetch = [&](int slot_i) {
+      const uint32_t rb = 4u * ld.rt + qq;
+      const uint8_t* vsrc = p.values + rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
+      uint8_t* slot = ring + slot_i * TC_SLOT_BYTES;
+      cp_async16(slot, vsrc);
+      cp_async16(slot + 512, vsrc + 512);
+      cp_async16(slot + 1024, p.meta + rb * mstride + (uint32_t)ld.g * 512u + lane * 16);
+      cp_async16(slot + 1536, p.scales + rb * sstride + (uint32_t)(ld.g >> 3) * 512u + lane * 16);
+      if (lane == 0) {
+        S.slot_rt[cw][slot_i] = ld.rt;
+        S.slot_g[cw][slot_i] = ld.g;
+      }
+      ld.advance(geo, TC_WG);
+    };
+#pragma unroll 1
+    for (int d = 0; d < TC_RING; ++d) {
+      if (d < nw) fetch(d);
+      cp_async_commit();
+    }
+    for (int i = 0; i < nw + TC_TS && ok; ++i) {
+      // read back tile i - TC_TS: its stage is the one tile i writes
+      const int j = i - TC_TS;
+      if (j >= 0) {
+        const int ts = j % TC_TS;
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.dfull[w][ts], (j / TC_TS) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        float d[B];
+        tmem_ld_wait<B>(tmem + lane_base + col_d(w, ts), d);
+        const float s = S.scale[w][ts][srow];
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[b] = fmaf(s, d[b], acc[b]);
+        const int rt = S.tinfo[w][ts][qq];
+        const int rt2 = j + 1 < nw ? S.tinfo[w][(j + 1) % TC_TS][qq] : -1;
+        if (rt2 != rt) {                            // last tile of this row tile in this warpgroup's range
+          const int row = rt * 128 + (int)srow;
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
+            acc[b] = 0.0f;
+          }
+        }
+      }
+      if (i >= nw) continue;
+      // convert tile i into tensor-memory stage i % TC_TS
+      const int ts = i % TC_TS, si = i % TC_RING;
+      uint8_t* slot = ring + si * TC_SLOT_BYTES;
+      cp_async_wait<TC_RING - 1>();
+      __syncwarp();                                 // lane 0's slot_rt / slot_g stores
+      const uint4 va = *reinterpret_cast<const uint4*>(slot);
+      const uint4 vb = *reinterpret_cast<const uint4*>(slot + 512);
+      const uint4 mm = *reinterpret_cast<const uint4*>(slot + 1024);
+      const int g = S.slot_g[cw][si], rt = S.slot_rt[cw][si];
+      const uint32_t sc16 = *reinterpret_cast<const uint16_t*>(slot + 1536 + 2 * (g & 7));
+      const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      uint32_t a[32];
+#pragma unroll
+      for (int wi = 0; wi < 8; ++wi) {
+        const uint32_t hi = vw[wi] >> 4;
+#pragma unroll
+        for (int by = 0; by < 4; ++by)
+          a[4 * wi + by] = code_pair<F16>(vw[wi], hi, (uint32_t)(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12)));
+      }
+      // META: this row's 32-bit code word of each K step holds groups 0..7 of
+      // it; the sparse MMA wants, in lane 16h + i, rows 16h + i and 16h + 8 + i
+      // side by side (16 bits each) for groups 0..3, and in lane 16h + 8 + i
+      // the same two rows for groups 4..7.
+      const uint32_t mw[4] = {mm.x, mm.y, mm.z, mm.w};
+      uint32_t me[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, mw[kk], 8);
+        me[kk] = prmt(mw[kk], o, sel_meta);
+      }
+      __syncwarp();                                 // all lanes read the slot's metadata
+      // refill the slot with tile i + TC_RING (after its bytes were used above)
+      if (i + TC_RING < nw) fetch(si);
+      cp_async_commit();
+      tmem_st32(tmem + lane_base + col_a(w, ts), a);
+      tmem_st8(tmem + lane_base + col_m(w, ts), me[0], me[1], 0u, 0u, me[2], me[3], 0u, 0u);
+      S.scale[w][ts][srow] = f16_bits_to_f32((uint16_t)sc16);
+      if (lane == 0) S.tinfo[w][ts][qq] = rt;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.afull[w][ts]);
+    }
+    cp_async_wait<0>();
+    if (!ok && lane == 0) set_error(p.err, CQL_ERR_TIMEOUT, 22);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  // complete only after the pre-kernel: the epilogue, which waits on this
+  // grid, then also sees the pre-kernel's CSR sums and adapter partials
+  if (p.has_pre && threadIdx.x == 0) pdl_wait();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host launch
+// ---------------------------------------------------------------------------
+bool decode_tc_eligible(const DecodeParams& p) {
+  return p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM && p.batch >= 1 && p.batch <= 16 &&
+         (p.xdt == CQL_DT_BF16 || p.xdt == CQL_DT_F16);
+}
+
+template <int B, bool F16>
+static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
+  TcGeom geo;
+  geo.n_rt = p.d.n_out / 128;
+  geo.G = p.d.k_in / 128;
+  geo.n_chunks = (geo.G + TC_KC - 1) / TC_KC;
+  geo.n_tiles = geo.n_rt * geo.G;
+  CUtensorMap mx;
+  if (!make_map_xchunk(&mx, p.x, (uint64_t)p.batch, (uint64_t)p.d.k_in, 16, 2 * TC_KC)) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(TcSmem) + 1024;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute((const void*)k_decode_tc<B, F16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  uint64_t grid = (uint64_t)device_sm_count();
+  if (grid > (uint64_t)geo.n_tiles) grid = (uint64_t)geo.n_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_decode_tc<B, F16>, mx, p, geo);
+}
+
+template <int B>
+static cudaError_t launch_tc_b(const DecodeParams& p, cudaStream_t st, bool pdl) {
+  return p.xdt == CQL_DT_F16 ? launch_tc<B, true>(p, st, pdl) : launch_tc<B, false>(p, st, pdl);
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int bpad, cudaStream_t st, bool pdl) {
+  switch (bpad) {
+    case 1: return launch_tc_b<1>(p, st, pdl);
+    case 2: return launch_tc_b<2>(p, st, pdl);
+    case 4: return launch_tc_b<4>(p, st, pdl);
+    case 8: return launch_tc_b<8>(p, st, pdl);
+    default: return launch_tc_b<16>(p, st, pdl);
+  }
+}
+
+}  // namespace cql

@@ -1,6 +1,8 @@
 // Parameter blocks and launch entry points shared by the host API and the
 // kernel translation units of libcql.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace cql {
@@ -97,7 +99,34 @@ struct ForwardWorkspace {
 };
 ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch);
 
+// The packed header matches the descriptor the call was made with.
+CQL_DEV bool header_ok(const DecodeParams& p) {
+  const uint32_t* h = reinterpret_cast<const uint32_t*>(p.header);
+  const int32_t* d = reinterpret_cast<const int32_t*>(p.header + 8);
+  return h[0] == 0x314C5143u /* "CQL1" */ && h[1] == CQL_VERSION && d[0] == p.d.n_out && d[1] == p.d.k_in &&
+         d[2] == p.d.mask && d[3] == p.d.codec && d[7] == p.d.rank;
+}
+
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+// Tensor-core decode of the main term (2:4 mask, int4 codes, bf16/f16 x).
+bool decode_tc_eligible(const DecodeParams& p);
+cudaError_t launch_decode_tc(const DecodeParams& p, int bpad, cudaStream_t st, bool pdl);
+int device_sm_count();
+
+// Tensor maps (tma_host.cu); false when the driver rejects the encoding.
+// 2-D 16-bit row-major matrix [rows][cols] (ld elements per row): boxes of
+// box_rows x 64 columns, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
+// 16-bit x [batch][k] seen as [k/64 column blocks][batch rows][64 columns]:
+// one box of box_blocks x box_rows x 64 lands as box_blocks consecutive
+// 128-byte-swizzled [box_rows][64] tiles (rows past the batch read as zero).
+bool make_map_xchunk(CUtensorMap* m, const void* x, uint64_t batch, uint64_t k, uint32_t box_rows, uint32_t box_blocks);
+// A row-interleaved plane seen as [n_blocks][block_bytes] (8-byte elements, no
+// swizzle): one box copies box_bytes from each of box_blocks consecutive row
+// blocks.
+bool make_map_rowblocks(CUtensorMap* m, const void* plane, uint64_t block_bytes, uint64_t n_blocks,
+                        uint32_t box_bytes, uint32_t box_blocks);
 
 // Prefill scratch (inside the forward workspace): byte offsets.
 struct PrefillLayout {
