@@ -37,7 +37,7 @@
 namespace cql {
 
 constexpr int kDecSmem = 220 * 1024;           // shared memory per CTA: tables + ring
-constexpr int kEpiThreads = 64;                 // epilogue block: two row blocks (one row group)
+constexpr int kEpiThreads = 128;                // epilogue block: four row blocks = one row group of 128
 
 constexpr uint32_t kMagic = 0x4B000000u;       // fp32 bit pattern of 2^23
 
@@ -517,38 +517,43 @@ __global__ void __launch_bounds__(U::kThreads, 1) k_decode(DecodeParams p, int r
 // codes and scales are read before waiting on the previous kernel; the
 // accumulator and t only after.
 // ---------------------------------------------------------------------------
+// At most 64 registers a thread, so that a block fits beside the tensor-core
+// decode kernel (640 threads x 88 registers) and prefetches its L codes (with
+// cp.async, into shared memory) while that kernel runs.
 template <int B>
-__global__ void __launch_bounds__(kEpiThreads, 1) k_epilogue(DecodeParams p, int kq) {
-  // u[b][j] = s_L[g][j] * t[b][j] for this block's row group g (a block's
-  // kEpiThreads rows lie in one group of 128)
-  __shared__ float us[B * 256];
+__global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
+  // dynamic shared memory: u[b][j] = s_L[g][j] t[b][j] (B x r floats), then the
+  // block's L codes, [32-column chunk m][thread] 16 bytes each
+  extern __shared__ __align__(16) uint8_t esm[];
   const int lane = threadIdx.x & 31;
   const int rb = blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5);
   const bool lowrank = p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK);
-  const bool active = rb < p.n_rb;
   const int N = p.d.n_out, r = p.d.rank;
   const int row = rb * 32 + lane;
-  const int g = (blockIdx.x * kEpiThreads) / kGroup;
-  uint4 lv[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {                     // rank <= 256: at most 8 chunks of 32
-    lv[m] = make_uint4(0u, 0u, 0u, 0u);
-    if (active && lowrank && 32 * m < r) lv[m] = ldg_stream(p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
-  }
+  const int g = (blockIdx.x * kEpiThreads) / kGroup;   // the block's rows lie in one group of 128
+  const int nch = (r + 31) / 32;
+  float* us = reinterpret_cast<float*>(esm);
+  uint8_t* lsm = esm + (size_t)B * p.r_pad * 4;
+  if (lowrank)
+    for (int m = 0; m < nch; ++m)
+      cp_async16(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16, p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
+  cp_async_commit();
   pdl_wait();                                       // main term (and pre-kernel) complete
   float acc[B];
 #pragma unroll
   for (int b = 0; b < B; ++b) {
     acc[b] = 0.0f;
-    if (active && b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
+    if (b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
   }
   if (lowrank) {
-    // every (b, j) of t: the K-slice partials, loaded four at a time
+    // every (b, j) of t: the accumulated t (slices == 0) or the sum of the
+    // pre-kernel's K-slice partials, loaded four at a time
     for (int i = threadIdx.x; i < B * r; i += kEpiThreads) {
       const int b = i / r, j = i - b * r;
+      float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
+      if (kq == 0) t0 = ld_cg_f32(p.t_final + (uint64_t)b * p.r_pad + j);
       const float* tp = p.t_part + (uint64_t)b * p.r_pad + j;
       const uint64_t st = (uint64_t)B * p.r_pad;
-      float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
       int k = 0;
       for (; k + 4 <= kq; k += 4) {
         t0 += ld_cg_f32(tp + (k + 0) * st);
@@ -561,30 +566,36 @@ __global__ void __launch_bounds__(kEpiThreads, 1) k_epilogue(DecodeParams p, int
     }
   }
   __syncthreads();
-  if (!active) return;
+  if (lowrank && kq == 0 && threadIdx.x == 0) {
+    // t_final is read by every block: the last block to have read it clears
+    // it (and the counter) for the next call
+    __threadfence();
+    if (atomicAdd(p.t_counter, 1u) == gridDim.x - 1) {
+      __threadfence();
+      for (int i = 0; i < B * p.r_pad; ++i) p.t_final[i] = 0.0f;
+      *p.t_counter = 0u;
+    }
+  }
 #pragma unroll
   for (int b = 0; b < B; ++b)
     if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
   if (lowrank) {
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      if (32 * m >= r) break;
-      const uint32_t wd[4] = {lv[m].x, lv[m].y, lv[m].z, lv[m].w};
-      float q[32];
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) q[jj] = (float)((int)((wd[jj >> 3] >> (4 * (jj & 7))) & 15u) - 8);
+    cp_async_wait<0>();
+    for (int m = 0; m < nch; ++m) {
+      const uint4 l4 = *reinterpret_cast<const uint4*>(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16);
+      const uint32_t wd[4] = {l4.x, l4.y, l4.z, l4.w};
       const int nj = min(32, r - 32 * m);           // 16 or 32
 #pragma unroll
-      for (int b = 0; b < B; ++b) {
-        const float* ub = us + b * r + 32 * m;
-        float a0 = 0.0f, a1 = 0.0f;
+      for (int jj = 0; jj < 32; jj += 4) {
+        if (jj >= nj) break;
+        const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
+        const float q0 = (float)((int)(wv & 15u) - 8), q1 = (float)((int)((wv >> 4) & 15u) - 8);
+        const float q2 = (float)((int)((wv >> 8) & 15u) - 8), q3 = (float)((int)((wv >> 12) & 15u) - 8);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) a0 = fmaf(q[jj], ub[jj], a0);
-        if (nj == 32) {
-#pragma unroll
-          for (int jj = 16; jj < 32; ++jj) a1 = fmaf(q[jj], ub[jj], a1);
+        for (int b = 0; b < B; ++b) {
+          const float4 u4 = *reinterpret_cast<const float4*>(us + b * r + 32 * m + jj);
+          acc[b] = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, acc[b]))));
         }
-        acc[b] += a0 + a1;
       }
     }
   }
@@ -781,6 +792,12 @@ static cudaError_t launch_main(const DecodeParams& p, cudaStream_t st, bool pdl)
   }
 }
 
+template <int B>
+static size_t epilogue_smem(const DecodeParams& p) {
+  const size_t r = (size_t)p.d.rank;
+  return (size_t)B * p.r_pad * 4 + ((r + 31) / 32) * kEpiThreads * 16;   // u, then the L codes
+}
+
 // pre (adapter partials, CSR rows) -> main term -> epilogue, each PDL-chained
 // to the one before it.
 template <int B>
@@ -793,6 +810,17 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
   const int n_csr = csr ? (p.d.n_out + 255) / 256 : 0;
   p.has_pre = (n_s1 + n_csr) > 0;
   cudaError_t e;
+  const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
+  if (main_on && decode_tc_eligible(p)) {
+    // tensor-core path: the main kernel also adds the CSR rows and t = R x
+    // (into t_final); the epilogue reads t_final directly (slices = 0)
+    p.has_pre = 0;
+    if ((e = launch_decode_tc(p, B, st, false)) != cudaSuccess) return e;
+    int zero = 0;
+    void* args0[2] = {&p, &zero};
+    const dim3 grid0((p.n_rb * 32 + kEpiThreads - 1) / kEpiThreads);
+    return launch_pdl((const void*)k_epilogue<B>, args0, grid0, dim3(kEpiThreads), epilogue_smem<B>(p), st, true);
+  }
   if (p.has_pre) {
     const size_t smem = (size_t)kS1Units * kGroup * B * 4;
     static bool attr_set = false;
@@ -804,15 +832,14 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
     k_pre<B><<<n_s1 + n_csr, 256, smem, st>>>(p, n_s1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
   if (main_on) {
-    e = decode_tc_eligible(p) ? launch_decode_tc(p, B, st, p.has_pre) : launch_main<B>(p, st, p.has_pre);
-    if (e != cudaSuccess) return e;
+    if ((e = launch_main<B>(p, st, p.has_pre)) != cudaSuccess) return e;
   }
   int kq_arg = kq;
   void* args[2] = {&p, &kq_arg};
   const dim3 grid((p.n_rb * 32 + kEpiThreads - 1) / kEpiThreads);
-  return launch_pdl((const void*)k_epilogue<B>, args, grid, dim3(kEpiThreads), 0, st, main_on || p.has_pre);
+  return launch_pdl((const void*)k_epilogue<B>, args, grid, dim3(kEpiThreads), epilogue_smem<B>(p), st,
+                    main_on || p.has_pre);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st) {

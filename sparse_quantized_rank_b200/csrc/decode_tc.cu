@@ -43,7 +43,7 @@ namespace {
 constexpr int TC_WG = 4;                          // converter warpgroups
 constexpr int TC_THREADS = 128 * (1 + TC_WG);     // warps 0..3 MMA issuers, then the warpgroups
 constexpr int TC_KC = 8;                          // scale groups per x chunk (1024 columns)
-constexpr int TC_RING = 4;                        // tiles in flight per converter warp (cp.async ring)
+constexpr int TC_RING = 3;                        // tiles in flight per converter warp (cp.async ring)
 constexpr int TC_TS = 2;                          // tensor-memory stages per converter warpgroup
 constexpr int TC_VAL_BYTES = 1024;                // codes of one 32-row block: 2 slabs
 constexpr int TC_META_BYTES = 512;                // META of one 32-row block: 1 slab
@@ -157,8 +157,83 @@ CQL_HD uint32_t tc_idesc(bool f16) {
   return (1u << 2) | (1u << 4) | (fmt << 7) | (fmt << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// Side work of the MMA issuer warps (all lanes), done before their MMA loops:
+// their first MMA waits for the first tile conversion anyway (it needs none
+// of the kernel's shared or tensor memory):
+//  * the CSR outliers (SqueezeLLM "Approach": the sparse part of the
+//    dense-and-sparse split) of this CTA's share of the rows, a thread per
+//    row, added into y_acc;
+//  * a share of t = deq(R_q) x (SLiM "Low-rank adapter quantization"): items
+//    of (32 R rows, 32 columns, all batch rows), a warp each, added into t_acc
+//    with the R group scale applied.
+template <int B>
+CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane) {
+  const int N = p.d.n_out, K = p.d.k_in;
+  if (p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR)) {
+    const int r0 = (int)((uint64_t)N * blockIdx.x / gridDim.x), r1 = (int)((uint64_t)N * (blockIdx.x + 1) / gridDim.x);
+    for (int row = r0 + iw * 32 + lane; row < r1; row += TC_WG * 32) {
+      int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
+      e0 = max(0, min(e0, (int)p.nnz));
+      e1 = max(e0, min(e1, (int)p.nnz));
+      if (e1 == e0) continue;
+      float acc[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+      for (int e = e0; e < e1; ++e) {
+        const int col = p.csr_col[e];
+        if (col >= K) continue;
+        const float v = f16_bits_to_f32(p.csr_val[e]);
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          if (b < p.batch) acc[b] = fmaf(v, to_f32_act(p.x, p.xdt, (uint64_t)b * K + col), acc[b]);
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * N + row, acc[b]);
+    }
+  }
+  if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK)) {
+    // item i goes to issuer warp i / gridDim.x (mod TC_WG) of CTA i % gridDim.x,
+    // so that the items spread over all CTAs before any warp gets a second one
+    const int items = (p.r_pad / 32) * (K / 32);
+    const int nwarps = gridDim.x * TC_WG;
+    for (int it = iw * gridDim.x + blockIdx.x; it < items; it += nwarps) {
+      const int s32 = it % (K / 32), rbr = it / (K / 32);
+      const int j = 32 * rbr + lane, u = s32 >> 2;
+      const uint4 q4 = ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
+      const float sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit32((uint32_t)j, 2u * u, p.rb.r_scales)));
+      float xv[B];                                  // x[b][32 s32 + lane]
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        xv[b] = 0.0f;
+        if (b < p.batch) {
+          const uint32_t xh = static_cast<const uint16_t*>(p.x)[(uint64_t)b * K + 32 * s32 + lane];
+          xv[b] = p.xdt == CQL_DT_BF16 ? bf16_bits_to_f32(xh) : f16_bits_to_f32(xh);
+        }
+      }
+      const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
+      float a[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) a[b] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float q = (float)((int)((wd[k >> 3] >> (4 * (k & 7))) & 15u) - 8);
+#pragma unroll
+        for (int b = 0; b < B; ++b) a[b] = fmaf(q, __shfl_sync(0xffffffffu, xv[b], k), a[b]);
+      }
+      if (j < p.d.rank) {
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          if (b < p.batch) atomicAdd(p.t_final + (uint64_t)b * p.r_pad + j, sc * a[b]);
+      }
+    }
+  }
+}
+
+// 88 registers per thread: 640 x 88 leaves room for one epilogue block (128
+// threads) to become resident beside this kernel and prefetch its operands.
 template <int B, bool F16>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __maxnreg__(88)
     k_decode_tc(const __grid_constant__ CUtensorMap tmX, DecodeParams p, TcGeom geo) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -205,20 +280,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // loads the x chunks (one 3-D TMA box each), one chunk ahead.  x chunk c
     // uses buffer c & 1; the chunks of the range are consecutive, so the
     // phase of a buffer follows from the chunk index.
+    TileIter first, last;
+    first.init(geo, t0);
+    last.init(geo, t1 - 1);
+    const int c0 = first.c, c1 = last.c;
+    if (warp == 0 && lane == 0 && n > 0) {
+      for (int c = c0; c <= min(c0 + 1, c1); ++c) {
+        mbar_expect_tx(&S.xfull[c & 1], TC_XCHUNK_BYTES);
+        tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
+      }
+    }
+    tc_side_work<B>(p, warp, lane);
+    __syncwarp();
     if (lane == 0 && n > 0) {
       const int w = warp;
       bool ok = true;
-      TileIter first, last;
-      first.init(geo, t0);
-      last.init(geo, t1 - 1);
-      const int c0 = first.c, c1 = last.c;
       auto phase = [&](int c) { return (uint32_t)(((c - c0) >> 1) & 1); };   // use index of buffer c & 1
-      if (w == 0) {
-        for (int c = c0; c <= min(c0 + 1, c1); ++c) {
-          mbar_expect_tx(&S.xfull[c & 1], TC_XCHUNK_BYTES);
-          tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
-        }
-      }
       int cur_c = -1, xc = -1;                      // chunk retired up to / chunk whose x is acquired
       uint32_t xb = 0;
       const uint32_t idesc = tc_idesc(F16);
@@ -380,9 +457,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
-  // complete only after the pre-kernel: the epilogue, which waits on this
-  // grid, then also sees the pre-kernel's CSR sums and adapter partials
-  if (p.has_pre && threadIdx.x == 0) pdl_wait();
 }
 
 }  // namespace
