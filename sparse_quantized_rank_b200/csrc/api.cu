@@ -117,11 +117,11 @@ ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch) {
   const uint64_t bp = batch <= CQL_MAX_DECODE_BATCH ? (uint64_t)padded_batch(batch) : 0;
   uint64_t pos = 0;
   w.err = pos;       pos = align256(pos + 8);
-  w.t_counter = pos; pos = align256(pos + 4);
+  w.t_counter = pos; pos = align256(pos + 8);    // [0] calls so far (tensor-core path), [1] this call's t buffer
   w.counters = pos;  pos = align256(pos + (n / 32) * 4);
   w.y_acc = pos;     pos = align256(pos + (batch <= CQL_MAX_DECODE_BATCH ? (uint64_t)batch * n * 4 : 0));
   w.t_part = pos;    pos = align256(pos + upr * bp * rpad * 4);
-  w.t_final = pos;   pos = align256(pos + bp * rpad * 4);
+  w.t_final = pos;   pos = align256(pos + 2 * bp * rpad * 4);   // two t buffers, alternating by call
   w.prefill = pos;
   if (batch > CQL_MAX_DECODE_BATCH) pos = align256(pos + prefill_layout(d, batch).total);
   w.total = pos;

@@ -154,6 +154,11 @@ CQL_DEV uint4 ldg_stream(const void* p) {
   return r;
 }
 CQL_DEV uint32_t ldg_u16(const uint8_t* p) { return __ldg(reinterpret_cast<const unsigned short*>(p)); }
+CQL_DEV uint32_t ld_cg_u32(const uint32_t* p) {
+  uint32_t r;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
 CQL_DEV float ld_cg_f32(const float* p) {
   float r;
   asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(r) : "l"(p));

@@ -546,12 +546,15 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     if (b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
   }
   if (lowrank) {
-    // every (b, j) of t: the accumulated t (slices == 0) or the sum of the
-    // pre-kernel's K-slice partials, loaded four at a time
+    // every (b, j) of t: the accumulated t (slices == 0: the buffer the main
+    // kernel named) or the sum of the pre-kernel's K-slice partials, loaded
+    // four at a time
+    const float* tfin = p.t_final + (kq == 0 ? (size_t)(ld_cg_u32(p.t_counter + 1) & 1u) * B * p.r_pad : 0);
+    if (kq == 0 && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(p.t_counter, 1u);   // next call: other buffer
     for (int i = threadIdx.x; i < B * r; i += kEpiThreads) {
       const int b = i / r, j = i - b * r;
       float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
-      if (kq == 0) t0 = ld_cg_f32(p.t_final + (uint64_t)b * p.r_pad + j);
+      if (kq == 0) t0 = ld_cg_f32(tfin + (uint64_t)b * p.r_pad + j);
       const float* tp = p.t_part + (uint64_t)b * p.r_pad + j;
       const uint64_t st = (uint64_t)B * p.r_pad;
       int k = 0;
@@ -566,16 +569,6 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     }
   }
   __syncthreads();
-  if (lowrank && kq == 0 && threadIdx.x == 0) {
-    // t_final is read by every block: the last block to have read it clears
-    // it (and the counter) for the next call
-    __threadfence();
-    if (atomicAdd(p.t_counter, 1u) == gridDim.x - 1) {
-      __threadfence();
-      for (int i = 0; i < B * p.r_pad; ++i) p.t_final[i] = 0.0f;
-      *p.t_counter = 0u;
-    }
-  }
 #pragma unroll
   for (int b = 0; b < B; ++b)
     if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;

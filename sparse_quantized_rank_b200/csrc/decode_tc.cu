@@ -169,6 +169,17 @@ CQL_HD uint32_t tc_idesc(bool f16) {
 template <int B>
 CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane) {
   const int N = p.d.n_out, K = p.d.k_in;
+  // t of this call accumulates in buffer (calls so far) & 1, which the call
+  // before cleared; clear the other one (the previous call's, whose epilogue
+  // is complete) for the next call
+  const uint32_t par = ld_cg_u32(p.t_counter) & 1u;
+  float* t_acc = p.t_final + (size_t)par * B * p.r_pad;
+  {
+    float* t_old = p.t_final + (size_t)(par ^ 1u) * B * p.r_pad;
+    const int tot = B * p.r_pad, per = (tot + gridDim.x - 1) / gridDim.x;
+    for (int i = blockIdx.x * per + iw * 32 + lane; i < min(tot, (int)(blockIdx.x + 1) * per); i += TC_WG * 32) t_old[i] = 0.0f;
+    if (blockIdx.x == 0 && iw == 0 && lane == 0) p.t_counter[1] = par;
+  }
   if (p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR)) {
     const int r0 = (int)((uint64_t)N * blockIdx.x / gridDim.x), r1 = (int)((uint64_t)N * (blockIdx.x + 1) / gridDim.x);
     for (int row = r0 + iw * 32 + lane; row < r1; row += TC_WG * 32) {
@@ -224,7 +235,7 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane) {
       if (j < p.d.rank) {
 #pragma unroll
         for (int b = 0; b < B; ++b)
-          if (b < p.batch) atomicAdd(p.t_final + (uint64_t)b * p.r_pad + j, sc * a[b]);
+          if (b < p.batch) atomicAdd(t_acc + (uint64_t)b * p.r_pad + j, sc * a[b]);
       }
     }
   }

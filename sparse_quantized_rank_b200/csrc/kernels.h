@@ -87,11 +87,12 @@ struct DecodeParams {
   int has_pre;       // a pre-kernel (adapter stage 1 and/or CSR rows) runs first, PDL-overlapped
   // workspace
   uint32_t* err;         // [2]
-  uint32_t* t_counter;   // [1]   low-rank stage-1 arrival counter
+  uint32_t* t_counter;   // [2]   tensor-core path: [0] calls so far (bumped by the epilogue), [1] the
+                         //       t buffer of the current call (written by the main kernel)
   float* y_acc;          // [batch][N]
   uint32_t* counters;    // [N/32]
   float* t_part;         // [upr][batch][r_pad]
-  float* t_final;        // [batch][r_pad]
+  float* t_final;        // [2][batch][r_pad]  tensor-core path: t = R x, the buffer alternating by call
 };
 
 struct ForwardWorkspace {
