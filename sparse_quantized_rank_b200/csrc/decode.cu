@@ -532,6 +532,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
   const int row = rb * 32 + lane;
   const int g = (blockIdx.x * kEpiThreads) / kGroup;   // the block's rows lie in one group of 128
   const int nch = (r + 31) / 32;
+  pdl_launch_dependents();                          // the next call's main kernel may start streaming
   float* us = reinterpret_cast<float*>(esm);
   uint8_t* lsm = esm + (size_t)B * p.r_pad * 4;
   if (lowrank)
@@ -808,7 +809,7 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
     // tensor-core path: the main kernel also adds the CSR rows and t = R x
     // (into t_final); the epilogue reads t_final directly (slices = 0)
     p.has_pre = 0;
-    if ((e = launch_decode_tc(p, B, st, false)) != cudaSuccess) return e;
+    if ((e = launch_decode_tc(p, B, st, true)) != cudaSuccess) return e;
     int zero = 0;
     void* args0[2] = {&p, &zero};
     const dim3 grid0((p.n_rb * 32 + kEpiThreads - 1) / kEpiThreads);

@@ -22,6 +22,10 @@
 // The scale is applied outside the MMA so that no dequantised weight is ever
 // rounded to 16 bits: the tensor cores multiply exact integers.
 //
+// Launched programmatically dependent on the previous kernel in the stream: the
+// weight tiles (inputs nobody writes) stream in before griddepcontrol.wait;
+// x, the accumulators and t are touched only after it.
+//
 // Roles (640 threads, one CTA per SM, persistent over a contiguous tile range):
 //   warps 0..3    MMA issuer of converter warpgroup 0..3 (one lane each);
 //                 warp 0 also allocates tensor memory and loads the x chunks
@@ -295,6 +299,9 @@ __global__ void __maxnreg__(88)
     first.init(geo, t0);
     last.init(geo, t1 - 1);
     const int c0 = first.c, c1 = last.c;
+    // x, the accumulators and t may be written by the kernels before this one
+    // (this kernel is launched early, programmatically dependent on them)
+    pdl_wait();
     if (warp == 0 && lane == 0 && n > 0) {
       for (int c = c0; c <= min(c0 + 1, c1); ++c) {
         mbar_expect_tx(&S.xfull[c & 1], TC_XCHUNK_BYTES);
@@ -366,6 +373,7 @@ __global__ void __maxnreg__(88)
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[b] = 0.0f;
     bool ok = true;
+    bool dep_done = false;                          // griddepcontrol.wait passed (before touching y_acc)
     // This warp's ring: lane l copies, and later reads back, only its own row's
     // 16-byte pieces (codes, META, the scale slab piece holding its group's
     // scale), so no cross-lane synchronisation is needed for them.
@@ -410,6 +418,10 @@ __global__ void __maxnreg__(88)
         const int rt2 = j + 1 < nw ? S.tinfo[w][(j + 1) % TC_TS][qq] : -1;
         if (rt2 != rt) {                            // last tile of this row tile in this warpgroup's range
           const int row = rt * 128 + (int)srow;
+          if (!dep_done) {
+            pdl_wait();
+            dep_done = true;
+          }
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
