@@ -535,9 +535,13 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
   pdl_launch_dependents();                          // the next call's main kernel may start streaming
   float* us = reinterpret_cast<float*>(esm);
   uint8_t* lsm = esm + (size_t)B * p.r_pad * 4;
-  if (lowrank)
+  uint16_t* ssm = reinterpret_cast<uint16_t*>(lsm + (size_t)nch * kEpiThreads * 16);   // s_L[g][0 .. r)
+  if (lowrank) {
     for (int m = 0; m < nch; ++m)
       cp_async16(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16, p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
+    for (int i = threadIdx.x; i < r / 2; i += kEpiThreads)   // r is a multiple of 16
+      cp_async4(ssm + 2 * i, p.l_scales + (uint64_t)g * r + 2 * i);
+  }
   cp_async_commit();
   pdl_wait();                                       // main term (and pre-kernel) complete
   float acc[B];
@@ -547,6 +551,8 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     if (b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
   }
   if (lowrank) {
+    cp_async_wait<0>();
+    __syncthreads();                                // the s_L row copied by other threads
     // every (b, j) of t: the accumulated t (slices == 0: the buffer the main
     // kernel named) or the sum of the pre-kernel's K-slice partials, loaded
     // four at a time
@@ -566,7 +572,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
         t3 += ld_cg_f32(tp + (k + 3) * st);
       }
       for (; k < kq; ++k) t0 += ld_cg_f32(tp + k * st);
-      us[i] = f16_bits_to_f32(p.l_scales[(uint64_t)g * r + j]) * ((t0 + t1) + (t2 + t3));
+      us[i] = f16_bits_to_f32(ssm[j]) * ((t0 + t1) + (t2 + t3));
     }
   }
   __syncthreads();
@@ -789,7 +795,7 @@ static cudaError_t launch_main(const DecodeParams& p, cudaStream_t st, bool pdl)
 template <int B>
 static size_t epilogue_smem(const DecodeParams& p) {
   const size_t r = (size_t)p.d.rank;
-  return (size_t)B * p.r_pad * 4 + ((r + 31) / 32) * kEpiThreads * 16;   // u, then the L codes
+  return (size_t)B * p.r_pad * 4 + ((r + 31) / 32) * kEpiThreads * 16 + (size_t)p.r_pad * 2;   // u, L codes, s_L
 }
 
 // pre (adapter partials, CSR rows) -> main term -> epilogue, each PDL-chained

@@ -170,8 +170,26 @@ CQL_HD uint32_t tc_idesc(bool f16) {
 //  * a share of t = deq(R_q) x (SLiM "Low-rank adapter quantization"): items
 //    of (32 R rows, 32 columns, all batch rows), a warp each, added into t_acc
 //    with the R group scale applied.
+// R codes and scale of the first R x item of a warp: weights, safe to read
+// before griddepcontrol.wait.
+struct SideFirst {
+  uint4 q4;
+  uint32_t sc;
+};
+CQL_DEV SideFirst tc_side_prefetch(const DecodeParams& p, int iw, int lane) {
+  SideFirst f{make_uint4(0u, 0u, 0u, 0u), 0u};
+  const int K = p.d.k_in;
+  const int it = iw * gridDim.x + blockIdx.x;
+  if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK) && it < (p.r_pad / 32) * (K / 32)) {
+    const int s32 = it % (K / 32), rbr = it / (K / 32);
+    f.q4 = ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
+    f.sc = ldg_u16(p.r_scales + rit32((uint32_t)(32 * rbr + lane), 2u * (s32 >> 2), p.rb.r_scales));
+  }
+  return f;
+}
+
 template <int B>
-CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane) {
+CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFirst& first) {
   const int N = p.d.n_out, K = p.d.k_in;
   // t of this call accumulates in buffer (calls so far) & 1, which the call
   // before cleared; clear the other one (the previous call's, whose epilogue
@@ -215,8 +233,9 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane) {
     for (int it = iw * gridDim.x + blockIdx.x; it < items; it += nwarps) {
       const int s32 = it % (K / 32), rbr = it / (K / 32);
       const int j = 32 * rbr + lane, u = s32 >> 2;
-      const uint4 q4 = ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
-      const float sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit32((uint32_t)j, 2u * u, p.rb.r_scales)));
+      const bool pre = it == iw * (int)gridDim.x + (int)blockIdx.x;   // the prefetched first item
+      const uint4 q4 = pre ? first.q4 : ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
+      const float sc = f16_bits_to_f32(pre ? first.sc : ldg_u16(p.r_scales + rit32((uint32_t)j, 2u * u, p.rb.r_scales)));
       float xv[B];                                  // x[b][32 s32 + lane]
 #pragma unroll
       for (int b = 0; b < B; ++b) {
@@ -299,6 +318,7 @@ __global__ void __maxnreg__(88)
     first.init(geo, t0);
     last.init(geo, t1 - 1);
     const int c0 = first.c, c1 = last.c;
+    const SideFirst side_first = tc_side_prefetch(p, warp, lane);
     // x, the accumulators and t may be written by the kernels before this one
     // (this kernel is launched early, programmatically dependent on them)
     pdl_wait();
@@ -308,7 +328,7 @@ __global__ void __maxnreg__(88)
         tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
       }
     }
-    tc_side_work<B>(p, warp, lane);
+    tc_side_work<B>(p, warp, lane, side_first);
     __syncwarp();
     if (lane == 0 && n > 0) {
       const int w = warp;
