@@ -68,7 +68,6 @@ CQL_HD uint32_t col_m(int w, int s) { return 128u * w + 96u + 8u * s; }
 
 struct TcSmem {
   uint8_t x[2][TC_XCHUNK_BYTES];                  // x chunks, 1024-byte aligned (128-byte swizzle atoms)
-  uint8_t bias[128 * 128];                        // constant A of the offset MMA (all elements equal)
   uint8_t ring[4 * TC_WG][TC_RING][TC_SLOT_BYTES];   // per converter warp: [values 1024][META 512][scales 512]
   int slot_rt[4 * TC_WG][TC_RING];                // row tile and group of each ring slot
   int slot_g[4 * TC_WG][TC_RING];
@@ -134,25 +133,27 @@ struct TileIter {
   }
 };
 
-// One 2:4 group's two codes u as exact 16-bit floats u + 128 (bf16) or
-// u + 1024 (f16).  'lo' holds the group's byte (low nibble: code of the first
-// kept column), 'hi' the same word shifted right by 4.  The byte permute puts
-// the two nibbles at bits 0 and 16; the LOP3 masks them and ORs in the
-// exponent of 128 (bf16: 0x4300) or 1024 (f16: 0x6400).  The offset, with the
-// code bias 8 (q = u - 8), is removed by a second MMA over the same kept
-// positions with a constant A of -136 (bf16) or -1032 (f16), so
-//   D = sum (u + 128) x - 136 sum x = sum q x     (bf16; f16 alike),
-// exact products in fp32 accumulation.
+// One 2:4 group's two codes u as exact 16-bit integers q = u - 8.  'lo'
+// holds the group's byte (low nibble: code of the first kept column), 'hi'
+// the same word shifted right by 4.  The byte permute puts the two nibbles at
+// bits 0 and 16; the LOP3 masks them and ORs in the exponent of 128 (bf16:
+// 0x4300, giving u + 128) or 1024 (f16: 0x6400, u + 1024); one packed
+// subtraction of 136 (1032) leaves q.  (Subtracting here costs one
+// instruction per pair; removing the offset with a second MMA over the same
+// metadata instead doubles the MMAs a tile issues, and MMA issue is the
+// scarcer resource.)
 template <bool F16>
 CQL_DEV uint32_t code_pair(uint32_t lo, uint32_t hi, uint32_t sel) {
   const uint32_t t = prmt(lo, hi, sel);
   uint32_t a;
   constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(t), "r"(0x000F000Fu), "r"(magic));
-  return a;
+  uint32_t q;
+  if (F16) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x64086408u));    // 1032
+  else asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x43084308u));      // 136
+  return q;
 }
-constexpr uint32_t kBiasBf16x2 = 0xC308C308u;     // -136, -136
-constexpr uint32_t kBiasF16x2 = 0xE408E408u;      // -1032, -1032
+
 
 // Instruction descriptor: sparse, D f32, A = B = bf16 (or f16), K-major,
 // M = 128, N = 16.
@@ -279,12 +280,6 @@ __global__ void __maxnreg__(88)
   const int t1 = (int)((uint64_t)geo.n_tiles * (blockIdx.x + 1) / gridDim.x);
   const int n = t1 - t0;
 
-  {
-    const uint32_t bv = F16 ? kBiasF16x2 : kBiasBf16x2;
-    for (int i = threadIdx.x; i < 128 * 128 / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(S.bias)[i] = make_uint4(bv, bv, bv, bv);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
-  }
   if (threadIdx.x == 0) {
     for (int w = 0; w < TC_WG; ++w)
       for (int s = 0; s < TC_TS; ++s) {
@@ -337,7 +332,6 @@ __global__ void __maxnreg__(88)
       int cur_c = -1, xc = -1;                      // chunk retired up to / chunk whose x is acquired
       uint32_t xb = 0;
       const uint32_t idesc = tc_idesc(F16);
-      const uint64_t dbias = smem_desc_sw128(smem_u32(S.bias));
       TileIter it;
       it.init(geo, t0 + w);
       for (int k = w; ok; k += TC_WG, it.advance(geo, TC_WG)) {
@@ -373,10 +367,7 @@ __global__ void __maxnreg__(88)
         tc_mma_sp_ta(d, a + 8, b1, m, idesc | 1u, 1u);
         tc_mma_sp_ta(d, a + 16, b2, m + 4, idesc, 1u);
         tc_mma_sp_ta(d, a + 24, b3, m + 4, idesc | 1u, 1u);
-        tc_mma_sp_ss(d, dbias, b0, m, idesc, 1u);
-        tc_mma_sp_ss(d, dbias, b1, m, idesc | 1u, 1u);
-        tc_mma_sp_ss(d, dbias, b2, m + 4, idesc, 1u);
-        tc_mma_sp_ss(d, dbias, b3, m + 4, idesc | 1u, 1u);
+
         tc_commit(&S.dfull[w][ts]);
       }
       if (!ok) set_error(p.err, CQL_ERR_TIMEOUT, 21);
