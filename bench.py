@@ -442,6 +442,7 @@ def extra_lines(torch, C, dev, stream, barrier):
                     "frac_of_measured_hbm": round(gbs / peak, 4), "bytes_per_step": b.bytes})
         del b
         torch.cuda.empty_cache()
+    out.append(stack_line(torch, C, dev, stream))
     tf_peak, _ = measured_tflops()
     for name in ("prefill_up", "prefill_down"):
         wl = workload(name)
@@ -459,6 +460,63 @@ def extra_lines(torch, C, dev, stream, barrier):
         del b
         torch.cuda.empty_cache()
     return out
+
+
+def stack_line(torch, C, dev, stream, passes=20):
+    """The 32-layer decode stack (LLaMA-7B shapes: q k v o 4096x4096, gate up
+    11008x4096, down 4096x11008; 2:4 int4 g128, rank 64, batch 1, each linear
+    with its own x): one pass = 224 forward calls, chained in stream order.
+    2.6 GB of packed weights, far beyond L2, so no rotation is needed.  The
+    weights are drawn on the device from the same distribution and per-linear
+    seeds as the workload recipe (timing only: values do not change the work)."""
+    from workloads import stack_layer_specs
+    specs = stack_layer_specs(32)
+    g = torch.Generator(device=dev)
+    calls, total_bytes, packed_bytes = [], 0, 0
+    for wl in specs:
+        g.manual_seed(wl.seed)
+        W = (torch.randn(wl.n, wl.k, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        L = torch.randn(wl.n, wl.rank, generator=g, device=dev) * 0.01
+        R = torch.randn(wl.rank, wl.k, generator=g, device=dev) * 0.01
+        layer = C.CompressedLinear(desc_from_workload(C, wl), W, L, R)
+        del W, L, R
+        x = torch.randn(1, wl.k, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(1, wl.n, dtype=torch.bfloat16, device=dev)
+        ws, wsb = layer.workspace(1)
+        calls.append((layer, x, y, ws, wsb))
+        total_bytes += algorithmic_bytes(layer.layout, 1, wl.n, wl.k)
+        packed_bytes += layer.layout.total_bytes
+    torch.cuda.synchronize()
+
+    def one_pass(s):
+        for layer, x, y, ws, wsb in calls:
+            C.compressed_linear_forward(layer.desc, layer.packed, x, C.CQL_DT_BF16, y, C.CQL_DT_BF16, 1, ws, wsb, s)
+
+    for _ in range(3):
+        one_pass(stream.cuda_stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        one_pass(torch.cuda.current_stream().cuda_stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(passes):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b) / 1e3)
+    peak, _ = measured_peaks()
+    best, med = min(times), float(np.median(times))
+    del graph, calls
+    torch.cuda.empty_cache()
+    return {"workload": "32-layer decode stack (224 linears, 2:4 int4 g128 r64, batch 1)",
+            "packed_MB": round(packed_bytes / 1e6, 1), "bytes_per_pass": total_bytes,
+            "us_per_pass_best": round(best * 1e6, 1), "us_per_pass_median": round(med * 1e6, 1),
+            "GB/s_median": round(total_bytes / med / 1e9, 1),
+            "frac_of_measured_hbm": round(total_bytes / med / 1e9 / peak, 4), "passes": passes}
 
 
 def main():
