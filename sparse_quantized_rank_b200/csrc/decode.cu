@@ -581,6 +581,14 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
   if (lowrank) {
     cp_async_wait<0>();
+    // independent partial sums per batch row (the FMA chain would otherwise
+    // run through all r terms one after the other)
+    constexpr int P = B <= 2 ? 4 : (B <= 4 ? 2 : 1);
+    float part[B][P];
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int k = 0; k < P; ++k) part[b][k] = 0.0f;
     for (int m = 0; m < nch; ++m) {
       const uint4 l4 = *reinterpret_cast<const uint4*>(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16);
       const uint32_t wd[4] = {l4.x, l4.y, l4.z, l4.w};
@@ -591,13 +599,19 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
         const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
         const float q0 = (float)((int)(wv & 15u) - 8), q1 = (float)((int)((wv >> 4) & 15u) - 8);
         const float q2 = (float)((int)((wv >> 8) & 15u) - 8), q3 = (float)((int)((wv >> 12) & 15u) - 8);
+        constexpr int kk = 0;
 #pragma unroll
         for (int b = 0; b < B; ++b) {
           const float4 u4 = *reinterpret_cast<const float4*>(us + b * r + 32 * m + jj);
-          acc[b] = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, acc[b]))));
+          float& a = part[b][(jj >> 2) % P + kk];
+          a = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, a))));
         }
       }
     }
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int k = 0; k < P; ++k) acc[b] += part[b][k];
   }
 #pragma unroll
   for (int b = 0; b < B; ++b)
