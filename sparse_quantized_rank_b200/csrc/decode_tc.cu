@@ -177,6 +177,13 @@ struct SideFirst {
   uint4 q4;
   uint32_t sc;
 };
+// Side workers per CTA: the 4 issuer warps for small batches; for 8 and more
+// batch rows the R x items are 8 to 16 times heavier and go to the 16
+// converter warps instead (at their first read-back, see the kernel).
+template <int B>
+constexpr int tc_side_workers() { return B >= 8 ? 4 * TC_WG : TC_WG; }
+
+template <int B>
 CQL_DEV SideFirst tc_side_prefetch(const DecodeParams& p, int iw, int lane) {
   SideFirst f{make_uint4(0u, 0u, 0u, 0u), 0u};
   const int K = p.d.k_in;
@@ -191,6 +198,7 @@ CQL_DEV SideFirst tc_side_prefetch(const DecodeParams& p, int iw, int lane) {
 
 template <int B>
 CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFirst& first) {
+  constexpr int NW = tc_side_workers<B>();
   const int N = p.d.n_out, K = p.d.k_in;
   // t of this call accumulates in buffer (calls so far) & 1, which the call
   // before cleared; clear the other one (the previous call's, whose epilogue
@@ -200,12 +208,12 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
   {
     float* t_old = p.t_final + (size_t)(par ^ 1u) * B * p.r_pad;
     const int tot = B * p.r_pad, per = (tot + gridDim.x - 1) / gridDim.x;
-    for (int i = blockIdx.x * per + iw * 32 + lane; i < min(tot, (int)(blockIdx.x + 1) * per); i += TC_WG * 32) t_old[i] = 0.0f;
+    for (int i = blockIdx.x * per + iw * 32 + lane; i < min(tot, (int)(blockIdx.x + 1) * per); i += NW * 32) t_old[i] = 0.0f;
     if (blockIdx.x == 0 && iw == 0 && lane == 0) p.t_counter[1] = par;
   }
   if (p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR)) {
     const int r0 = (int)((uint64_t)N * blockIdx.x / gridDim.x), r1 = (int)((uint64_t)N * (blockIdx.x + 1) / gridDim.x);
-    for (int row = r0 + iw * 32 + lane; row < r1; row += TC_WG * 32) {
+    for (int row = r0 + iw * 32 + lane; row < r1; row += NW * 32) {
       int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
       e0 = max(0, min(e0, (int)p.nnz));
       e1 = max(e0, min(e1, (int)p.nnz));
@@ -230,7 +238,7 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
     // item i goes to issuer warp i / gridDim.x (mod TC_WG) of CTA i % gridDim.x,
     // so that the items spread over all CTAs before any warp gets a second one
     const int items = (p.r_pad / 32) * (K / 32);
-    const int nwarps = gridDim.x * TC_WG;
+    const int nwarps = gridDim.x * NW;
     for (int it = iw * gridDim.x + blockIdx.x; it < items; it += nwarps) {
       const int s32 = it % (K / 32), rbr = it / (K / 32);
       const int j = 32 * rbr + lane, u = s32 >> 2;
@@ -313,7 +321,8 @@ __global__ void __maxnreg__(88)
     first.init(geo, t0);
     last.init(geo, t1 - 1);
     const int c0 = first.c, c1 = last.c;
-    const SideFirst side_first = tc_side_prefetch(p, warp, lane);
+    constexpr bool issuer_side = tc_side_workers<B>() == TC_WG;
+    const SideFirst side_first = issuer_side ? tc_side_prefetch<B>(p, warp, lane) : SideFirst{};
     // x, the accumulators and t may be written by the kernels before this one
     // (this kernel is launched early, programmatically dependent on them)
     pdl_wait();
@@ -323,7 +332,7 @@ __global__ void __maxnreg__(88)
         tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
       }
     }
-    tc_side_work<B>(p, warp, lane, side_first);
+    if (issuer_side) tc_side_work<B>(p, warp, lane, side_first);
     __syncwarp();
     if (lane == 0 && n > 0) {
       const int w = warp;
@@ -412,9 +421,18 @@ __global__ void __maxnreg__(88)
       if (d < nw) fetch(d);
       cp_async_commit();
     }
+    constexpr bool conv_side = tc_side_workers<B>() != TC_WG;
+    bool side_done = !conv_side;
+    const SideFirst side_first = conv_side ? tc_side_prefetch<B>(p, cw, lane) : SideFirst{};
     for (int i = 0; i < nw + TC_TS && ok; ++i) {
       // read back tile i - TC_TS: its stage is the one tile i writes
       const int j = i - TC_TS;
+      if (conv_side && j == 0) {                    // the first MMA results are some way off
+        pdl_wait();
+        tc_side_work<B>(p, cw, lane, side_first);
+        dep_done = true;
+        side_done = true;
+      }
       if (j >= 0) {
         const int ts = j % TC_TS;
         ok = __all_sync(0xffffffffu, mbar_wait(&S.dfull[w][ts], (j / TC_TS) & 1));
@@ -485,6 +503,10 @@ __global__ void __maxnreg__(88)
       if (lane == 0) mbar_arrive(&S.afull[w][ts]);
     }
     cp_async_wait<0>();
+    if (!side_done) {                               // no tile here, or stopped early: the side work still runs
+      pdl_wait();
+      tc_side_work<B>(p, cw, lane, side_first);
+    }
     if (!ok && lane == 0) set_error(p.err, CQL_ERR_TIMEOUT, 22);
   }
   tc_fence_before();
