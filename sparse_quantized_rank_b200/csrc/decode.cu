@@ -558,10 +558,20 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     // four at a time
     const float* tfin = p.t_final + (kq == 0 ? (size_t)(ld_cg_u32(p.t_counter + 1) & 1u) * B * p.r_pad : 0);
     if (kq == 0 && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(p.t_counter, 1u);   // next call: other buffer
-    for (int i = threadIdx.x; i < B * r; i += kEpiThreads) {
+    if (kq == 0) {
+      // a thread's columns j, all batch rows: B loads in flight before any is used
+      for (int j = threadIdx.x; j < r; j += kEpiThreads) {
+        float v[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) v[b] = b < p.batch ? ld_cg_f32(tfin + (uint64_t)b * p.r_pad + j) : 0.0f;
+        const float sl = f16_bits_to_f32(ssm[j]);
+#pragma unroll
+        for (int b = 0; b < B; ++b) us[b * r + j] = sl * v[b];
+      }
+    }
+    for (int i = threadIdx.x; kq > 0 && i < B * r; i += kEpiThreads) {
       const int b = i / r, j = i - b * r;
       float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
-      if (kq == 0) t0 = ld_cg_f32(tfin + (uint64_t)b * p.r_pad + j);
       const float* tp = p.t_part + (uint64_t)b * p.r_pad + j;
       const uint64_t st = (uint64_t)B * p.r_pad;
       int k = 0;
@@ -581,37 +591,41 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
     if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
   if (lowrank) {
     cp_async_wait<0>();
-    // independent partial sums per batch row (the FMA chain would otherwise
-    // run through all r terms one after the other)
-    constexpr int P = B <= 2 ? 4 : (B <= 4 ? 2 : 1);
-    float part[B][P];
+    // batch rows in groups of up to 4 (bounded live registers), each with
+    // independent partial sums (the FMA chain would otherwise run through all
+    // r terms one after the other)
+    constexpr int BG = B < 4 ? B : 4;
+    constexpr int P = B <= 2 ? 4 : 2;
 #pragma unroll
-    for (int b = 0; b < B; ++b)
+    for (int b0 = 0; b0 < B; b0 += BG) {
+      float part[BG][P];
 #pragma unroll
-      for (int k = 0; k < P; ++k) part[b][k] = 0.0f;
-    for (int m = 0; m < nch; ++m) {
-      const uint4 l4 = *reinterpret_cast<const uint4*>(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16);
-      const uint32_t wd[4] = {l4.x, l4.y, l4.z, l4.w};
-      const int nj = min(32, r - 32 * m);           // 16 or 32
+      for (int bb = 0; bb < BG; ++bb)
 #pragma unroll
-      for (int jj = 0; jj < 32; jj += 4) {
-        if (jj >= nj) break;
-        const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
-        const float q0 = (float)((int)(wv & 15u) - 8), q1 = (float)((int)((wv >> 4) & 15u) - 8);
-        const float q2 = (float)((int)((wv >> 8) & 15u) - 8), q3 = (float)((int)((wv >> 12) & 15u) - 8);
-        constexpr int kk = 0;
+        for (int k = 0; k < P; ++k) part[bb][k] = 0.0f;
+      for (int m = 0; m < nch; ++m) {
+        const uint4 l4 = *reinterpret_cast<const uint4*>(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16);
+        const uint32_t wd[4] = {l4.x, l4.y, l4.z, l4.w};
+        const int nj = min(32, r - 32 * m);         // 16 or 32
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const float4 u4 = *reinterpret_cast<const float4*>(us + b * r + 32 * m + jj);
-          float& a = part[b][(jj >> 2) % P + kk];
-          a = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, a))));
+        for (int jj = 0; jj < 32; jj += 4) {
+          if (jj >= nj) break;
+          const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
+          const float q0 = (float)((int)(wv & 15u) - 8), q1 = (float)((int)((wv >> 4) & 15u) - 8);
+          const float q2 = (float)((int)((wv >> 8) & 15u) - 8), q3 = (float)((int)((wv >> 12) & 15u) - 8);
+#pragma unroll
+          for (int bb = 0; bb < BG; ++bb) {
+            const float4 u4 = *reinterpret_cast<const float4*>(us + (b0 + bb) * r + 32 * m + jj);
+            float& a = part[bb][(jj >> 2) % P];
+            a = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, a))));
+          }
         }
       }
+#pragma unroll
+      for (int bb = 0; bb < BG; ++bb)
+#pragma unroll
+        for (int k = 0; k < P; ++k) acc[b0 + bb] += part[bb][k];
     }
-#pragma unroll
-    for (int b = 0; b < B; ++b)
-#pragma unroll
-      for (int k = 0; k < P; ++k) acc[b] += part[b][k];
   }
 #pragma unroll
   for (int b = 0; b < B; ++b)
