@@ -165,6 +165,11 @@ CQL_DEV float ld_cg_f32(const float* p) {
   return r;
 }
 
+// Signed int4 code (stored u = q + 8) in bits 0..3 of y as the float q,
+// without an integer-to-float conversion: with u in the low mantissa bits of
+// 2^23 the float is 2^23 + u exactly.
+CQL_DEV float nib_f32(uint32_t y) { return __uint_as_float((y & 0x0Fu) | 0x4B000000u) - 8388616.0f; }
+
 // Programmatic dependent launch controls (no-ops without a PDL edge).
 // 16-byte asynchronous global -> shared copies (LSU path), grouped per thread.
 CQL_DEV void cp_async16(void* smem_dst, const void* gsrc) {

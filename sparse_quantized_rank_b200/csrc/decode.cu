@@ -611,8 +611,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
         for (int jj = 0; jj < 32; jj += 4) {
           if (jj >= nj) break;
           const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
-          const float q0 = (float)((int)(wv & 15u) - 8), q1 = (float)((int)((wv >> 4) & 15u) - 8);
-          const float q2 = (float)((int)((wv >> 8) & 15u) - 8), q3 = (float)((int)((wv >> 12) & 15u) - 8);
+          const float q0 = nib_f32(wv), q1 = nib_f32(wv >> 4), q2 = nib_f32(wv >> 8), q3 = nib_f32(wv >> 12);
 #pragma unroll
           for (int bb = 0; bb < BG; ++bb) {
             const float4 u4 = *reinterpret_cast<const float4*>(us + (b0 + bb) * r + 32 * m + jj);

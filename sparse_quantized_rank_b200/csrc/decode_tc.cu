@@ -54,6 +54,15 @@ constexpr int TC_META_BYTES = 512;                // META of one 32-row block: 1
 constexpr int TC_SLOT_BYTES = TC_VAL_BYTES + TC_META_BYTES + 512;   // one row block of one tile (+ scale slab)
 constexpr int TC_XBOX_BYTES = 16 * 64 * 2;        // TMA box: 16 rows x 64 columns of 16-bit x
 constexpr int TC_XCHUNK_BYTES = TC_KC * 2 * TC_XBOX_BYTES;
+// Up to 8 batch rows the box holds 8 rows (one 1 KB swizzle atom): the MMA
+// still reads 16 rows (N = 16), its rows 8..15 falling on the next box, but
+// they only reach accumulator columns 8..15, which are never read.
+template <int B>
+constexpr int tc_xrows() { return B <= 8 ? 8 : 16; }
+template <int B>
+constexpr int tc_xbox_bytes() { return tc_xrows<B>() * 64 * 2; }
+template <int B>
+constexpr int tc_xchunk_bytes() { return TC_KC * 2 * tc_xbox_bytes<B>(); }
 
 // Tensor-memory columns of converter warpgroup w (512 allocated, 128 each):
 //   A (compressed codes) stage s: 128 w + 32 s          (32 columns)
@@ -328,7 +337,7 @@ __global__ void __maxnreg__(88)
     pdl_wait();
     if (warp == 0 && lane == 0 && n > 0) {
       for (int c = c0; c <= min(c0 + 1, c1); ++c) {
-        mbar_expect_tx(&S.xfull[c & 1], TC_XCHUNK_BYTES);
+        mbar_expect_tx(&S.xfull[c & 1], tc_xchunk_bytes<B>());
         tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
       }
     }
@@ -351,7 +360,7 @@ __global__ void __maxnreg__(88)
             if (w == 0 && cur_c + 2 <= c1) {        // chunk cur_c + 2 reuses that buffer
               const int cn = cur_c + 2, b = cn & 1;
               if (!mbar_wait(&S.xempty[b], phase(cn) ^ 1)) { ok = false; break; }
-              mbar_expect_tx(&S.xfull[b], TC_XCHUNK_BYTES);
+              mbar_expect_tx(&S.xfull[b], tc_xchunk_bytes<B>());
               tma_load_3d(S.x[b], &tmX, &S.xfull[b], 0, 0, cn * 2 * TC_KC);
             }
           }
@@ -368,10 +377,11 @@ __global__ void __maxnreg__(88)
         const int i = k / TC_WG, ts = i % TC_TS;
         if (!mbar_wait(&S.afull[w][ts], (i / TC_TS) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t xg = xb + (uint32_t)(2 * it.gl) * TC_XBOX_BYTES;
+        constexpr uint32_t XBOX = tc_xbox_bytes<B>();
+        const uint32_t xg = xb + (uint32_t)(2 * it.gl) * XBOX;
         const uint32_t d = tmem + col_d(w, ts), a = tmem + col_a(w, ts), m = tmem + col_m(w, ts);
         const uint64_t b0 = smem_desc_sw128(xg), b1 = smem_desc_sw128(xg + 64);
-        const uint64_t b2 = smem_desc_sw128(xg + TC_XBOX_BYTES), b3 = smem_desc_sw128(xg + TC_XBOX_BYTES + 64);
+        const uint64_t b2 = smem_desc_sw128(xg + XBOX), b3 = smem_desc_sw128(xg + XBOX + 64);
         tc_mma_sp_ta(d, a, b0, m, idesc, 0u);
         tc_mma_sp_ta(d, a + 8, b1, m, idesc | 1u, 1u);
         tc_mma_sp_ta(d, a + 16, b2, m + 4, idesc, 1u);
@@ -420,6 +430,14 @@ __global__ void __maxnreg__(88)
     for (int d = 0; d < TC_RING; ++d) {
       if (d < nw) fetch(d);
       cp_async_commit();
+    }
+    if (B <= 4) {
+      // small batches: no conversion before the dependency resolves (the
+      // conversions would take issue slots from the previous call's epilogue,
+      // which runs beside this kernel on the same SMs); from 8 batch rows on,
+      // converting ahead is worth more
+      pdl_wait();
+      dep_done = true;
     }
     constexpr bool conv_side = tc_side_workers<B>() != TC_WG;
     bool side_done = !conv_side;
@@ -533,7 +551,7 @@ static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
   geo.n_chunks = (geo.G + TC_KC - 1) / TC_KC;
   geo.n_tiles = geo.n_rt * geo.G;
   CUtensorMap mx;
-  if (!make_map_xchunk(&mx, p.x, (uint64_t)p.batch, (uint64_t)p.d.k_in, 16, 2 * TC_KC)) return cudaErrorInvalidValue;
+  if (!make_map_xchunk(&mx, p.x, (uint64_t)p.batch, (uint64_t)p.d.k_in, tc_xrows<B>(), 2 * TC_KC)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(TcSmem) + 1024;
   static bool attr_set = false;
   if (!attr_set) {
