@@ -217,9 +217,11 @@ cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t s
  *             aligned.
  *   y         device [batch][N], y_dt = CQL_DT_F32, F16 or BF16, 16-byte
  *             aligned; fp32 accumulation, one final round to y_dt.
- *   batch     1..16 runs the CUDA-core decode GEMV (bandwidth bound); larger
- *             batches run the tcgen05 tensor-core prefill GEMM, which is
- *             implemented for 2:4 int4 layers (others: CQL_ERR_UNSUPPORTED).
+ *   batch     1..16 runs the decode path: sparse tcgen05 MMAs for 2:4 int4
+ *             layers with fp16/bf16 x, a CUDA-core GEMV for the other codecs
+ *             and masks; larger batches run the tcgen05 tensor-core prefill
+ *             GEMM, which is implemented for 2:4 int4 layers (others:
+ *             CQL_ERR_UNSUPPORTED).
  *   workspace device, >= cql_workspace_size bytes, 256-byte aligned, zeroed
  *             by cql_workspace_init before its first use with a given layer
  *             and batch (the forward leaves it ready for the next call with

@@ -24,6 +24,11 @@ REDUCED = {
     "int3_dense": workload("down_unstructured", n=256, k=384, mask="none", rank=0),
     "lut4_lr": workload("lut_dense_sparse", n=384, k=768, codec="lut4", rank=32),
     "bitmap_int4_csr": workload("down_unstructured", n=256, k=896, codec="int4", outlier_frac=0.002, rank=16),
+    # tensor-core path with every term: CSR rows and R x as side work, a K
+    # that ends in a one-group x chunk (33 groups), rank 48 (a half adapter
+    # chunk), fp16 x; 16 row tiles x 33 groups = 528 tiles, so CTAs hold
+    # several tiles and cross row tiles and x chunks
+    "int4_2of4_csr_ragged": workload("mlp_up", n=2048, k=4224, outlier_frac=0.002, rank=48, x_dtype="f16"),
 }
 FULL = {
     "mlp_up": workload("mlp_up"),
@@ -70,6 +75,7 @@ def test_pack_bit_exact(name, cuda_dev):
     ("int3_dense", (1, 2)),
     ("lut4_lr", (1, 4)),
     ("bitmap_int4_csr", (1, 9)),
+    ("int4_2of4_csr_ragged", (1, 3, 8, 13)),
     ("mlp_up", (1, 4, 16)),
     ("lut_dense_sparse", (1, 8)),
     ("down_unstructured", (1, 2, 4, 8, 16)),
@@ -87,7 +93,7 @@ def test_forward_matches_oracle(name, batches, cuda_dev):
 
 
 @pytest.mark.parametrize("name", ["tiny", "mlp_up_small", "lut_small", "down_small", "int4_dense_csr",
-                                  "lut4_lr", "bitmap_int4_csr"])
+                                  "lut4_lr", "bitmap_int4_csr", "int4_2of4_csr_ragged"])
 def test_each_term_alone(name, cuda_dev):
     """Every term checked on its own scale (a bug in the small adapter or CSR
     term cannot hide inside the tolerance of the sum)."""
