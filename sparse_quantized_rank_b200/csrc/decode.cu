@@ -589,7 +589,30 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
 #pragma unroll
   for (int b = 0; b < B; ++b)
     if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
-  if (lowrank) {
+  if (lowrank && B >= 8) {
+    cp_async_wait<0>();
+    // 8 and more batch rows: every code is converted once per 8 batch rows,
+    // each row's sum running in its own accumulator (the 8 chains are
+    // independent of one another)
+#pragma unroll
+    for (int b0 = 0; b0 < B; b0 += 8)
+    for (int m = 0; m < nch; ++m) {
+      const uint4 l4 = *reinterpret_cast<const uint4*>(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16);
+      const uint32_t wd[4] = {l4.x, l4.y, l4.z, l4.w};
+      const int nj = min(32, r - 32 * m);           // 16 or 32
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 4) {
+        if (jj >= nj) break;
+        const uint32_t wv = wd[jj >> 3] >> (4 * (jj & 7));
+        const float q0 = nib_f32(wv), q1 = nib_f32(wv >> 4), q2 = nib_f32(wv >> 8), q3 = nib_f32(wv >> 12);
+#pragma unroll
+        for (int b = b0; b < b0 + 8; ++b) {
+          const float4 u4 = *reinterpret_cast<const float4*>(us + b * r + 32 * m + jj);
+          acc[b] = fmaf(q0, u4.x, fmaf(q1, u4.y, fmaf(q2, u4.z, fmaf(q3, u4.w, acc[b]))));
+        }
+      }
+    }
+  } else if (lowrank) {
     cp_async_wait<0>();
     // batch rows in groups of up to 4 (bounded live registers), each with
     // independent partial sums (the FMA chain would otherwise run through all
