@@ -6,8 +6,9 @@
 // A tile is 128 weight rows x one scale group (128 columns).  Per tile:
 //   * each converter warp fetches its 32-row block's packed bytes (two code
 //     slabs and one META slab, 16 bytes per lane each) with cp.async, several
-//     tiles ahead; x (the MMA's B operand, batch padded to 16 rows with zeros)
-//     arrives in chunks of 1024 columns, one 3-D TMA box per chunk;
+//     tiles ahead; x (the MMA's B operand, batch padded with zeros to the
+//     box's 8 or 16 rows) arrives in chunks of 1024 columns, one 3-D TMA box
+//     per chunk;
 //   * a converter warpgroup (lanes = rows, as the planes are laid out) turns
 //     the 64 kept codes of each row into exact bf16/f16 integers and writes
 //     them straight into tensor memory (compressed A, 32 columns), and writes
