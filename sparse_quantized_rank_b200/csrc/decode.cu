@@ -658,8 +658,8 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
 // pre-kernel, PDL primary of the decode kernel:
 //  * blocks [0, n_s1): low-rank stage 1, t = deq(R_q) x.  Block (R row block,
 //    K slice of up to 8 units): a warp per unit, partial sums reduced in shared
-//    memory, per-slice partials; the last block to finish sums the slices in
-//    a fixed order into t_final (deterministic).
+//    memory, one partial per K slice in t_part; the epilogue sums the slices
+//    in a fixed order (deterministic).
 //  * blocks [n_s1, ..): the CSR outliers, a thread per output row, added into
 //    the fp32 accumulator (SqueezeLLM "Approach": the sparse part of the
 //    dense-and-sparse decomposition).
