@@ -206,6 +206,76 @@ def test_uniform_textbook_rtn_special_case():
     assert (q2 == q).all()
 
 
+def _rtn_exact(v: Fraction, s: Fraction, qmax: int) -> int:
+    """Round v / s to the nearest integer, ties to even, then clamp: exact
+    rational arithmetic, independent of the oracle's floating point."""
+    if s == 0:
+        return 0
+    t = v / s
+    fl = math.floor(t)
+    rem = t - fl
+    q = fl + 1 if (rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1)) else fl
+    return max(-qmax, min(qmax, q))
+
+
+def test_uniform_scale_excludes_outliers():
+    """With CSR outliers the group scale comes from the remaining entries:
+    s = fp16(alpha * max |w| over the non-outlier entries / qmax); an outlier
+    itself still gets a code (clamped to the grid edge), which the CSR value
+    corrects (SqueezeLLM "Approach": the outliers leave the dense part so that
+    its range narrows)."""
+    rng = np.random.default_rng(99)
+    for bits in (4, 3):
+        qmax = 2 ** (bits - 1) - 1
+        w = rng.standard_normal((3, 256)) * 0.02
+        ex = np.zeros_like(w, dtype=bool)
+        # the true maximum of three groups is an excluded outlier (x40 and
+        # negative in one of them); one group has two outliers
+        for (n, k, f) in ((0, 5, 40.0), (1, 130, -40.0), (2, 77, 35.0), (2, 78, 30.0)):
+            w[n, k] = f * 0.02
+            ex[n, k] = True
+        q, s = O.quantize_uniform(w, bits, 0.9, exclude=ex)
+        alpha = Fraction(float(np.float32(0.9)))
+        for n in range(3):
+            for g in range(2):
+                seg = range(128 * g, 128 * g + 128)
+                amax = max(abs(Fraction(float(w[n, j]))) for j in seg if not ex[n, j])
+                s_exact = fp16_round_exact(alpha * amax / qmax)
+                assert Fraction(float(s[n, g])) == s_exact, (bits, n, g)
+                for j in seg:
+                    assert int(q[n, j]) == _rtn_exact(Fraction(float(w[n, j])), s_exact, qmax), (bits, n, j)
+        # the excluded entries sit at the grid edge with their own sign
+        for (n, k) in zip(*np.nonzero(ex)):
+            assert int(q[n, k]) == int(np.sign(w[n, k])) * qmax
+        # without the exclusion the outlier would set the scale instead
+        _, s_in = O.quantize_uniform(w, bits, 0.9)
+        assert s_in[0, 0] > s[0, 0]
+
+
+def test_compress_passes_outliers_to_the_uniform_scale():
+    """compress() with a uniform codec and a CSR matrix takes each group's
+    scale without the selected outliers, and dense + CSR reproduces every
+    outlier to within half an fp16 ulp of the CSR value."""
+    wl = workload("mlp_up", n=128, k=256, mask="none", outlier_frac=0.004, rank=0, seed=31)
+    inp = make_layer_inputs(wl)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"])
+    w = inp["w"].astype(np.float64)
+    k = w.shape[1]
+    out = set(int(i) for i in parts["out_idx"])
+    assert len(out) == math.floor(float(np.float32(0.004)) * 128 * 256)
+    alpha = Fraction(float(np.float32(wl.clip_alpha)))
+    for n in range(0, 128, 9):
+        for g in range(2):
+            vals = [abs(Fraction(float(w[n, j]))) for j in range(128 * g, 128 * g + 128) if n * k + j not in out]
+            assert Fraction(float(parts["scales"][n, g])) == fp16_round_exact(alpha * max(vals) / 7)
+    rp, col, val = parts["csr_row_ptr"], parts["csr_col"], parts["csr_val"]
+    rows = np.repeat(np.arange(128), np.diff(rp))
+    for r_, c_, v_ in zip(rows, col, val):
+        assert r_ * k + c_ in out
+        assert abs(v_ + parts["w_dense"][r_, c_] - w[r_, c_]) <= half_ulp16(v_)
+
+
 def test_uniform_zero_group():
     w = np.zeros((1, 256))
     w[0, 200] = 0.3
@@ -348,7 +418,7 @@ def _brute_forward(parts, desc, x):
     for b in range(x.shape[0]):
         for i in range(n):
             y[b, i] = math.fsum(W[i][j] * float(x[b, j]) for j in range(k))
-    return y
+    return y, np.array(W)
 
 
 @pytest.mark.parametrize("name,over", [
@@ -362,8 +432,12 @@ def test_forward_matches_brute_force(name, over):
     d = O.desc_for(wl)
     parts = O.compress(d, inp["w"], inp["L"], inp["R"])
     y = O.forward(parts, inp["x"])
-    yb = _brute_forward(parts, d, inp["x"])
+    yb, Wb = _brute_forward(parts, d, inp["x"])
     assert O.rel_err(y, yb) < 1e-12
+    # the explicit dense reconstruction W_hat = deq(Q (.) M) + S + deq(L) deq(R)
+    # is the brute-force matrix, element by element
+    Wd = O.dense_reconstruction(parts)
+    assert np.abs(Wd - Wb).max() <= 1e-15 * max(np.abs(Wb).max(), 1.0)
 
 
 def test_forward_linear_and_term_isolation():
