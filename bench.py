@@ -86,6 +86,14 @@ def algorithmic_bytes(layout, batch, n, k, x_bytes=2, y_bytes=2):
     return planes + batch * k * x_bytes + batch * n * y_bytes
 
 
+def algorithmic_bytes_oracle(O, wl, batch):
+    """The same byte count from the oracle's copy of the packed layout (the
+    reference arm touches no GPU)."""
+    lay = O.packed_layout(O.desc_for(wl))
+    planes = sum(int(lay["len"][i]) for i in range(12) if i not in (PLANE_HEADER, PLANE_VOFF))
+    return planes + batch * wl.k * 2 + batch * wl.n * 2
+
+
 def desc_from_workload(C, wl):
     mask = {"2:4": C.CQL_MASK_2_4, "bitmap50": C.CQL_MASK_BITMAP50, "none": C.CQL_MASK_NONE}[wl.mask]
     codec = {"int4": C.CQL_CODEC_INT4_SYM, "int3": C.CQL_CODEC_INT3_SYM, "lut3": C.CQL_CODEC_LUT3_ROW,
@@ -230,21 +238,31 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    import oracle as O
     from workloads import workload
     wl = workload(args.workload)
     gbs, steps, rows, threads, dt = cpu_oracle_rate(wl, args.batch, seconds=60.0, steps=args.steps,
                                                     warmup=args.warmup)
     sample = f"{rows} of {wl.n} output rows per step (fp64 oracle forward), {steps} steps"
+    cfg = bench_config(wl, args.batch, int(os.environ.get("WORLD_SIZE", "1")))
+    cfg["bytes_per_step"] = int(algorithmic_bytes_oracle(O, wl, args.batch))
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": steps, "warmup": args.warmup, "ms_per_step": dt / max(steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": wl_name(wl, args.batch)},
+        "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def bench_config(wl, batch, world):
+    """The "config" object of the JSON line, identical for both arms."""
+    return {"workload": wl_name(wl, batch), "bytes_per_step": None,
+            "l2": "inputs larger than L2: packed copies rotating over more than 2.2x the L2 size",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def wl_name(wl, batch):
@@ -260,13 +278,14 @@ def wl_name(wl, batch):
 class Bench:
     """One packed layer, rotated over enough copies to defeat L2."""
 
-    def __init__(self, wl, batch, dev, torch, C):
+    def __init__(self, wl, batch, dev, torch, C, flags=0):
         from workloads import make_layer_inputs
         self.torch, self.C, self.wl, self.batch = torch, C, wl, batch
         inp = make_layer_inputs(wl, max_batch=batch)
         W, L, R, x = device_inputs(torch, inp, wl, dev)
         self.desc = desc_from_workload(C, wl)
         self.layer = C.CompressedLinear(self.desc, W, L, R)
+        self.desc.flags = flags                     # forward-only flags (the packed header keeps 0)
         del W, L, R
         torch.cuda.synchronize()
         self.layout = self.layer.layout
@@ -316,6 +335,10 @@ class Bench:
             sampler.start()
             time.sleep(0.3)
         with torch.cuda.stream(stream):
+            # one untimed replay queued right before the timed ones: the GPU
+            # idled while the clock sampler started, and the timed region (a
+            # few hundred microseconds for short runs) must not start cold
+            graph.replay()
             start.record(stream)
             for _ in range(n_rep):
                 graph.replay()
@@ -411,10 +434,8 @@ def run_cql(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl_name(wl, args.batch), "bytes_per_step": b.bytes,
-                   "l2": f"inputs larger than L2: {b.ncopy} rotating packed copies "
-                         f"({b.ncopy * b.layout.total_bytes / 1e6:.0f} MB)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": dict(bench_config(wl, args.batch, world), bytes_per_step=b.bytes),
+        "l2_rotation": f"{b.ncopy} rotating packed copies ({b.ncopy * b.layout.total_bytes / 1e6:.0f} MB)",
         "pct_of_8TBs": value / world / 8000.0 * 100,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
@@ -435,6 +456,15 @@ def run_cql(args):
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                                 "sample": f"fp64 oracle forward over {rows} of {wl.n} rows, {steps} steps, "
                                           f"{dt:.1f} s"}
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                gbs1, steps1, rows1, _, dt1 = cpu_oracle_rate(wl, args.batch, args.cpu_seconds / 2)
+            line["cpu_baseline_1thread"] = {
+                "value": gbs1, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                "sample": f"fp64 oracle forward over {rows1} of {wl.n} rows, {steps1} steps, {dt1:.1f} s"}
+        except ImportError:
+            pass
     if not args.no_extra:
         line["extra"] = extra_lines(torch, C, dev, stream, barrier)
     if world > 1:
@@ -450,7 +480,7 @@ def extra_lines(torch, C, dev, stream, barrier):
     from workloads import workload
     out = []
     peak, _ = measured_peaks()
-    for name, batch in (("tiny", 1), ("mlp_up", 4), ("mlp_up", 16), ("lut_dense_sparse", 1),
+    for name, batch in (("mlp_up", 1), ("tiny", 1), ("mlp_up", 4), ("mlp_up", 16), ("lut_dense_sparse", 1),
                         ("lut_dense_sparse", 8), ("down_unstructured", 1), ("down_unstructured", 16)):
         wl = workload(name)
         b = Bench(wl, batch, dev, torch, C)
@@ -458,6 +488,18 @@ def extra_lines(torch, C, dev, stream, barrier):
         gbs = b.bytes * 20000 / total / 1e9
         out.append({"workload": wl_name(wl, batch), "GB/s": round(gbs, 1), "us_per_step": round(total / 20000 * 1e6, 3),
                     "frac_of_measured_hbm": round(gbs / peak, 4), "bytes_per_step": b.bytes})
+        del b
+        torch.cuda.empty_cache()
+    # the same layer decoded on the CUDA cores (the design the tensor-core
+    # decode replaced for 2:4 int4 layers), for comparison
+    for batch in (1, 16):
+        wl = workload("mlp_up")
+        b = Bench(wl, batch, dev, torch, C, flags=C.CQL_FLAG_CUDA_CORE)
+        total, per, _ = b.timed(20000, 200, stream)
+        gbs = b.bytes * 20000 / total / 1e9
+        out.append({"workload": wl_name(wl, batch) + " (CUDA-core decode)", "GB/s": round(gbs, 1),
+                    "us_per_step": round(total / 20000 * 1e6, 3), "frac_of_measured_hbm": round(gbs / peak, 4),
+                    "bytes_per_step": b.bytes})
         del b
         torch.cuda.empty_cache()
     out.append(stack_line(torch, C, dev, stream))

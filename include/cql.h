@@ -145,6 +145,15 @@ enum {
 #define CQL_FLAG_NO_MAIN 0x1u
 #define CQL_FLAG_NO_CSR 0x2u
 #define CQL_FLAG_NO_LOWRANK 0x4u
+/* Test only: the tensor-core decode skips loading x, so that its bounded
+ * waits on x run out (after ~10 ms instead of seconds); the call then
+ * completes with CQL_ERR_TIMEOUT in the device error word and y undefined,
+ * and the next call on the same workspace is clean.  No copy or MMA is left
+ * in flight: nothing that waits on x has started any. */
+#define CQL_FLAG_DEBUG_SKIP_X 0x100u
+/* Decode on the CUDA cores even where the tensor-core decode applies (2:4
+ * int4 layers); for comparing the two designs on the same layer. */
+#define CQL_FLAG_CUDA_CORE 0x200u
 
 /* Layer descriptor, 64 bytes, stored verbatim in the packed header. */
 typedef struct cql_desc {
@@ -205,6 +214,13 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
  * Host only. */
 cql_status cql_workspace_size(const cql_desc* desc, int32_t batch, uint64_t* bytes);
 
+/* Reads before the previous kernel completes.  The forward's first kernel is
+ * launched programmatically dependent on the kernel that precedes it on the
+ * stream and reads the packed weights (never x, y or the workspace) before
+ * waiting for that kernel to complete.  So the kernel immediately before a
+ * forward must not write the packed buffer; pack_compressed_weight ends with
+ * an operation that makes a forward launched right after it safe. */
+
 /* Zero a forward workspace (required once before its first use; the forward
  * leaves the parts it reuses zeroed again when it completes). */
 cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t stream);
@@ -247,13 +263,17 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
  *   All calls share the array, and each call first clears (memset on its
  *   stream) the part of it that it uses: calls that overlap on the GPU race,
  *   so order them on one stream.  Device errors are recorded in the array's
- *   error word and are not reported back by this entry point. */
+ *   error word; read them with cql_get_device_status(NULL, stream, &st). */
 cql_status compressed_linear_forward_noalloc(const cql_desc* desc, const void* packed, const void* x,
                                              cql_dtype x_dt, void* y, cql_dtype y_dt, int32_t batch,
                                              cql_stream_t stream);
 
 /* Wait for the stream, then read and clear the device error word of a
- * workspace: *out = CQL_OK or the cql_status a kernel recorded. */
+ * workspace: *out = CQL_OK or the cql_status a kernel recorded.
+ *   workspace  a forward workspace, or NULL for the fixed scratch array of
+ *              compressed_linear_forward_noalloc on the current device (each
+ *              no-workspace call clears that word when it starts, so this
+ *              reports the most recent such call; CQL_OK if none ran). */
 cql_status cql_get_device_status(void* workspace, cql_stream_t stream, cql_status* out);
 
 #ifdef __cplusplus

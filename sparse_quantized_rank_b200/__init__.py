@@ -27,6 +27,8 @@ CQL_MASK_NONE, CQL_MASK_2_4, CQL_MASK_BITMAP50 = 0, 1, 2
 CQL_CODEC_INT4_SYM, CQL_CODEC_INT3_SYM, CQL_CODEC_LUT3_ROW, CQL_CODEC_LUT4_ROW = 0, 1, 2, 3
 CQL_DT_F32, CQL_DT_F16, CQL_DT_BF16 = 0, 1, 2
 CQL_FLAG_NO_MAIN, CQL_FLAG_NO_CSR, CQL_FLAG_NO_LOWRANK = 1, 2, 4
+CQL_FLAG_DEBUG_SKIP_X = 0x100
+CQL_FLAG_CUDA_CORE = 0x200
 CQL_NPLANES = 12
 CQL_MAX_DECODE_BATCH = 16
 
@@ -176,6 +178,8 @@ def compressed_linear_forward_noalloc(desc, packed, x, x_dt, y, y_dt, batch, str
 
 
 def cql_get_device_status(workspace, stream=None) -> int:
+    """Device error word of a workspace (None: the fixed scratch of the
+    no-workspace entry point on the current device)."""
     v = ctypes.c_int()
     _check(lib().cql_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(v)), "cql_get_device_status")
     return int(v.value)

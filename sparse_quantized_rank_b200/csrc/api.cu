@@ -292,7 +292,15 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
 }
 
 cql_status cql_get_device_status(void* workspace, cql_stream_t stream, cql_status* out) {
-  if (workspace == nullptr || out == nullptr) return CQL_ERR_ARG;
+  if (out == nullptr) return CQL_ERR_ARG;
+  if (workspace == nullptr) {
+    // the fixed scratch of the no-workspace entry point on the current device
+    workspace = noalloc_scratch_current_device();
+    if (workspace == nullptr) {                     // no such call has run here
+      *out = CQL_OK;
+      return CQL_OK;
+    }
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint32_t w[2] = {0, 0};
   if (cudaMemcpyAsync(w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess) return CQL_ERR_CUDA;

@@ -777,15 +777,13 @@ static cudaError_t launch_unit(DecodeParams p, int unit_bytes, int extra_bytes, 
   p.n_tiles = (p.upr + ktu - 1) / ktu;
   const int ring_off = ktu * unit_bytes + extra_bytes;
   const size_t smem = (size_t)ring_off + ring;
-  static bool attr_set = false;       // once per instantiation: allow the opt-in maximum
-  if (!attr_set) {
+  static std::atomic<uint64_t> attr_done{0};   // per instantiation and device: allow the opt-in maximum
+  {
     int dev = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    cudaError_t e = cudaFuncSetAttribute((const void*)k_decode<U, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         optin > 0 ? optin : (int)smem);
+    cudaError_t e = ensure_smem_attr(attr_done, (const void*)k_decode<U, B>, optin > 0 ? optin : (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   uint64_t grid = (uint64_t)device_sm_count();
   if (grid > p.n_units) grid = p.n_units;
@@ -861,7 +859,7 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
   p.has_pre = (n_s1 + n_csr) > 0;
   cudaError_t e;
   const bool main_on = !(p.flags & CQL_FLAG_NO_MAIN);
-  if (main_on && decode_tc_eligible(p)) {
+  if (main_on && decode_tc_eligible(p) && !(p.flags & CQL_FLAG_CUDA_CORE)) {
     // tensor-core path: the main kernel also adds the CSR rows and t = R x
     // (into t_final); the epilogue reads t_final directly (slices = 0)
     p.has_pre = 0;
@@ -873,12 +871,8 @@ static cudaError_t launch_decode_b(const DecodeParams& p0, cudaStream_t st) {
   }
   if (p.has_pre) {
     const size_t smem = (size_t)kS1Units * kGroup * B * 4;
-    static bool attr_set = false;
-    if (!attr_set) {
-      e = cudaFuncSetAttribute((const void*)k_pre<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    if ((e = ensure_smem_attr(attr_done, (const void*)k_pre<B>, (int)smem)) != cudaSuccess) return e;
     k_pre<B><<<n_s1 + n_csr, 256, smem, st>>>(p, n_s1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -292,7 +292,7 @@ __global__ void __maxnreg__(88)
   TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();                          // let the epilogue kernel get resident
-  if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
+  const long long wlim = (p.flags & CQL_FLAG_DEBUG_SKIP_X) ? kTcDebugWaitCycles : kTcWaitCycles;
 
   const int t0 = (int)((uint64_t)geo.n_tiles * blockIdx.x / gridDim.x);
   const int t1 = (int)((uint64_t)geo.n_tiles * (blockIdx.x + 1) / gridDim.x);
@@ -336,7 +336,9 @@ __global__ void __maxnreg__(88)
     // x, the accumulators and t may be written by the kernels before this one
     // (this kernel is launched early, programmatically dependent on them)
     pdl_wait();
-    if (warp == 0 && lane == 0 && n > 0) {
+    // the header too may have been written by the kernel before this one
+    if (blockIdx.x == 0 && threadIdx.x == 0 && !header_ok(p)) set_error(p.err, CQL_ERR_FORMAT, 1);
+    if (warp == 0 && lane == 0 && n > 0 && !(p.flags & CQL_FLAG_DEBUG_SKIP_X)) {
       for (int c = c0; c <= min(c0 + 1, c1); ++c) {
         mbar_expect_tx(&S.xfull[c & 1], tc_xchunk_bytes<B>());
         tma_load_3d(S.x[c & 1], &tmX, &S.xfull[c & 1], 0, 0, c * 2 * TC_KC);
@@ -360,7 +362,7 @@ __global__ void __maxnreg__(88)
             tc_commit(&S.xempty[cur_c & 1]);        // free once this issuer's MMAs on it finish
             if (w == 0 && cur_c + 2 <= c1) {        // chunk cur_c + 2 reuses that buffer
               const int cn = cur_c + 2, b = cn & 1;
-              if (!mbar_wait(&S.xempty[b], phase(cn) ^ 1)) { ok = false; break; }
+              if (!mbar_wait(&S.xempty[b], phase(cn) ^ 1, wlim)) { ok = false; break; }
               mbar_expect_tx(&S.xfull[b], tc_xchunk_bytes<B>());
               tma_load_3d(S.x[b], &tmX, &S.xfull[b], 0, 0, cn * 2 * TC_KC);
             }
@@ -370,13 +372,13 @@ __global__ void __maxnreg__(88)
         if (!ok || k >= n) break;
         if (c != xc) {
           const int b = c & 1;
-          if (!mbar_wait(&S.xfull[b], phase(c))) { ok = false; break; }
+          if (!mbar_wait(&S.xfull[b], phase(c), wlim)) { ok = false; break; }
           xb = smem_u32(S.x[b]);
           xc = c;
           tc_fence_after();
         }
         const int i = k / TC_WG, ts = i % TC_TS;
-        if (!mbar_wait(&S.afull[w][ts], (i / TC_TS) & 1)) { ok = false; break; }
+        if (!mbar_wait(&S.afull[w][ts], (i / TC_TS) & 1, wlim)) { ok = false; break; }
         tc_fence_after();
         constexpr uint32_t XBOX = tc_xbox_bytes<B>();
         const uint32_t xg = xb + (uint32_t)(2 * it.gl) * XBOX;
@@ -454,7 +456,7 @@ __global__ void __maxnreg__(88)
       }
       if (j >= 0) {
         const int ts = j % TC_TS;
-        ok = __all_sync(0xffffffffu, mbar_wait(&S.dfull[w][ts], (j / TC_TS) & 1));
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.dfull[w][ts], (j / TC_TS) & 1, wlim));
         if (!ok) break;
         tc_fence_after();
         float d[B];
@@ -554,13 +556,9 @@ static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
   CUtensorMap mx;
   if (!make_map_xchunk(&mx, p.x, (uint64_t)p.batch, (uint64_t)p.d.k_in, tc_xrows<B>(), 2 * TC_KC)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(TcSmem) + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute((const void*)k_decode_tc<B, F16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = ensure_smem_attr(attr_done, (const void*)k_decode_tc<B, F16>, (int)smem);
+  if (e != cudaSuccess) return e;
   uint64_t grid = (uint64_t)device_sm_count();
   if (grid > (uint64_t)geo.n_tiles) grid = (uint64_t)geo.n_tiles;
   cudaLaunchConfig_t cfg = {};

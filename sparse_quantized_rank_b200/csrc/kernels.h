@@ -3,6 +3,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace cql {
@@ -109,6 +111,23 @@ CQL_DEV bool header_ok(const DecodeParams& p) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+// Device address of compressed_linear_forward_noalloc's scratch array on the
+// current device (nullptr before its first call there).
+void* noalloc_scratch_current_device();
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) applies to the device that
+// is current when it runs, so the opt-in is made once per (kernel, device):
+// 'done' holds one bit per device index (a repeated call is harmless).
+inline cudaError_t ensure_smem_attr(std::atomic<uint64_t>& done, const void* f, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Tensor-core decode of the main term (2:4 mask, int4 codes, bf16/f16 x).
 bool decode_tc_eligible(const DecodeParams& p);

@@ -56,6 +56,18 @@ void* scratch_for_current_device(cql_status* st) {
 
 }  // namespace
 
+namespace cql {
+// The scratch array's device address on the current device, or nullptr when
+// no no-workspace call has run on it yet (cql_get_device_status reads its
+// error word when passed no workspace).
+void* noalloc_scratch_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  return g_scratch_ptr[dev];
+}
+}  // namespace cql
+
 extern "C" {
 
 cql_status compressed_linear_forward_noalloc(const cql_desc* desc, const void* packed, const void* x,

@@ -483,6 +483,13 @@ __global__ void k_adapter_L(PackParams p) {
 // ---------------------------------------------------------------------------
 // host-side launch sequence
 // ---------------------------------------------------------------------------
+// Last operation of every pack: an empty kernel launched with an ordinary
+// (full) stream dependency.  The forward's first kernel is launched
+// programmatically dependent on whatever kernel precedes it and reads the
+// packed weights before waiting for that kernel; with this kernel last, every
+// byte of the packed buffer was written before that kernel even started.
+__global__ void k_pack_done() {}
+
 static cudaError_t set_smem(const void* f, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -550,6 +557,7 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
     const int nL = (N / kGroup) * (p.d.rank / 2);
     k_adapter_L<<<(nL + 127) / 128, 128, 0, st>>>(p);
   }
+  k_pack_done<<<1, 32, 0, st>>>();
   return cudaGetLastError();
 }
 

@@ -473,13 +473,9 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   cudaError_t e = check_gemm_regs();
   if (e != cudaSuccess) return e;
 
-  static bool attr_set = false;
+  static std::atomic<uint64_t> attr_done{0};
   const size_t smem = sizeof(PfSmem) + 1024;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute((const void*)k_pf_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if ((e = ensure_smem_attr(attr_done, (const void*)k_pf_gemm, (int)smem)) != cudaSuccess) return e;
   const uint64_t nw = (uint64_t)N * G;
   if (p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM)
     k_pf_dequant_w24<<<(unsigned)(((uint64_t)p.n_rb * G + kDqWarps - 1) / kDqWarps), kDqWarps * 32, 0, st>>>(

@@ -9,6 +9,8 @@
 namespace cql {
 
 constexpr long long kTcWaitCycles = 4000000000ll;   // a wait longer than this is an error
+// Wait limit under CQL_FLAG_DEBUG_SKIP_X (a test makes a wait run out on purpose).
+constexpr long long kTcDebugWaitCycles = 20000000ll;
 // Each try_wait may suspend the thread this long (it resumes as soon as the
 // phase completes), so that waiting warps do not spin on the issue slots.
 constexpr uint32_t kTcSuspendNs = 1000000u;
@@ -29,7 +31,7 @@ CQL_DEV void mbar_arrive(uint64_t* bar) {
 // kTcWaitCycles SM clock cycles have passed (about 2 s at the boost clock,
 // longer at lower clocks); the caller records an error and winds down.  The
 // bound is kept with the SM cycle counter, which is cheap to read.
-CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kTcWaitCycles) {
   const uint32_t a = smem_u32(bar);
   long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
@@ -43,7 +45,7 @@ CQL_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     if (done) return true;
     if (it == 0) t0 = clock64();
-    else if ((it & 63) == 0 && clock64() - t0 > kTcWaitCycles) return false;
+    else if ((it & 7) == 0 && clock64() - t0 > limit) return false;
   }
 }
 CQL_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {

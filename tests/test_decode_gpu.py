@@ -9,8 +9,8 @@ import pytest
 
 import oracle as O
 import sparse_quantized_rank_b200 as C
-from tests.gpu_util import Case, check_close
-from workloads import workload
+from tests.gpu_util import Case, c_desc, check_close, device_inputs
+from workloads import make_layer_inputs, stack_layer_specs, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -35,6 +35,12 @@ FULL = {
     "lut_dense_sparse": workload("lut_dense_sparse"),
     "down_unstructured": workload("down_unstructured"),
 }
+# The other shapes of the 32-layer LLaMA-7B decode stack (2:4 int4 g128,
+# rank 64, bf16, batch 1), drawn by the stack's own per-linear seeds: q
+# (4096x4096), gate (11008x4096) and down (4096x11008) of layer 0.
+_STACK0 = {wl.name.split(".")[-1]: wl for wl in stack_layer_specs(1)}
+STACK = {f"stack_{k}": _STACK0[k] for k in ("q", "gate", "down")}
+FULL.update(STACK)
 
 _cache = {}
 
@@ -79,6 +85,9 @@ def test_pack_bit_exact(name, cuda_dev):
     ("mlp_up", (1, 4, 16)),
     ("lut_dense_sparse", (1, 8)),
     ("down_unstructured", (1, 2, 4, 8, 16)),
+    ("stack_q", (1,)),
+    ("stack_gate", (1,)),
+    ("stack_down", (1,)),
 ])
 def test_forward_matches_oracle(name, batches, cuda_dev):
     import torch
@@ -141,3 +150,72 @@ def test_corrupt_header_reported(cuda_dev):
         case.layer.packed[:4] = saved
     case.forward(1, torch.float32)
     assert case.layer.device_status(1) == C.CQL_OK
+
+
+def test_layers_chained_without_sync(cuda_dev):
+    """Several different layers called back to back on one stream with no
+    synchronisation in between (each forward is launched programmatically
+    dependent on the kernel before it, which belongs to another layer); every
+    output is then checked against the oracle."""
+    import torch
+    names = ["mlp_up_small", "int4_2of4_csr_ragged", "down_small", "tiny", "mlp_up_small"]
+    cases = [get_case(n, cuda_dev) for n in names]
+    torch.cuda.synchronize()
+    outs = []
+    for case, b in zip(cases, (1, 3, 2, 1, 16)):
+        outs.append((case, b, case.forward(b, torch.float32)))
+    torch.cuda.synchronize()
+    for case, b, y in outs:
+        check_close(y, case.reference(b), "f32", what=f"chained {case.wl.name} B={b}")
+        assert case.layer.device_status(b) == C.CQL_OK
+
+
+def test_pack_then_forward_without_sync(cuda_dev):
+    """Packing and the first forward on one stream with no synchronisation in
+    between: the forward must see every packed byte (its first kernel reads
+    weights before waiting for the kernel that precedes it)."""
+    import torch
+    for wl, b in ((workload("mlp_up", n=1024, k=2048, seed=41), 1),
+                  (workload("mlp_up", n=512, k=1024, seed=42, outlier_frac=0.002, rank=32), 4)):
+        inp = make_layer_inputs(wl, max_batch=b)
+        od = O.desc_for(wl)
+        parts = O.compress(od, inp["w"], inp["L"], inp["R"])
+        W, L, R, x = device_inputs(inp, wl, cuda_dev)
+        torch.cuda.synchronize()
+        layer = C.CompressedLinear(c_desc(od), W, L, R)      # pack: queued, not waited for
+        y = layer.forward(x[:b].contiguous(), out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        check_close(y, O.forward(parts, inp["x"][:b].astype(np.float64)), "f32", what=f"pack+forward {wl.n}x{wl.k}")
+        assert np.array_equal(layer.packed.cpu().numpy(), O.pack_bytes(od, parts))
+        assert layer.device_status(b) == C.CQL_OK
+
+
+@pytest.mark.parametrize("batch", [1, 16])
+def test_bounded_wait_runs_out_and_is_reported(batch, cuda_dev):
+    """A call whose x load is skipped (test flag) lets the tensor-core decode's
+    bounded waits on x run out: the call completes, the device error word says
+    CQL_ERR_TIMEOUT, and the next ordinary call on the same workspace is clean
+    and correct.  No GPU fault is involved: nothing that waits on x has issued
+    a copy or an MMA when the waits give up."""
+    import torch
+    case = get_case("mlp_up_small", cuda_dev)
+    case.forward(batch, torch.float32)
+    assert case.layer.device_status(batch) == C.CQL_OK
+    case.forward(batch, torch.float32, flags=C.CQL_FLAG_DEBUG_SKIP_X)
+    assert case.layer.device_status(batch) == C.CQL_ERR_TIMEOUT
+    y = case.forward(batch, torch.float32)
+    assert case.layer.device_status(batch) == C.CQL_OK
+    check_close(y, case.reference(batch), "f32", what=f"after timeout B={batch}")
+
+
+@pytest.mark.parametrize("name,batches", [("mlp_up_small", (1, 4, 16)), ("int4_2of4_csr_ragged", (1, 13))])
+def test_cuda_core_decode_of_2of4_int4(name, batches, cuda_dev):
+    """The CUDA-core decode of a 2:4 int4 layer (selected by flag; the
+    tensor-core decode is the default for these layers) against the oracle."""
+    import torch
+    case = get_case(name, cuda_dev)
+    for b in batches:
+        y = case.forward(b, torch.float32, flags=C.CQL_FLAG_CUDA_CORE)
+        torch.cuda.synchronize()
+        check_close(y, case.reference(b), "f32", what=f"{name} cuda-core B={b}")
+        assert case.layer.device_status(b) == C.CQL_OK
