@@ -147,9 +147,10 @@ enum {
 #define CQL_FLAG_NO_LOWRANK 0x4u
 /* Test only: the tensor-core decode skips loading x, so that its bounded
  * waits on x run out (after ~10 ms instead of seconds); the call then
- * completes with CQL_ERR_TIMEOUT in the device error word and y undefined,
- * and the next call on the same workspace is clean.  No copy or MMA is left
- * in flight: nothing that waits on x has started any. */
+ * completes with CQL_ERR_TIMEOUT in the device error word and y undefined.
+ * No copy or MMA is left in flight: nothing that waits on x has started any.
+ * As after any device error, the workspace must be initialised again
+ * (cql_workspace_init) before its next use. */
 #define CQL_FLAG_DEBUG_SKIP_X 0x100u
 /* Decode on the CUDA cores even where the tensor-core decode applies (2:4
  * int4 layers); for comparing the two designs on the same layer. */
@@ -269,7 +270,9 @@ cql_status compressed_linear_forward_noalloc(const cql_desc* desc, const void* p
                                              cql_stream_t stream);
 
 /* Wait for the stream, then read and clear the device error word of a
- * workspace: *out = CQL_OK or the cql_status a kernel recorded.
+ * workspace: *out = CQL_OK or the cql_status a kernel recorded.  After an
+ * error the rest of the workspace is in an undefined state: initialise it
+ * again with cql_workspace_init before the next forward that uses it.
  *   workspace  a forward workspace, or NULL for the fixed scratch array of
  *              compressed_linear_forward_noalloc on the current device (each
  *              no-workspace call clears that word when it starts, so this

@@ -203,6 +203,8 @@ def test_bounded_wait_runs_out_and_is_reported(batch, cuda_dev):
     assert case.layer.device_status(batch) == C.CQL_OK
     case.forward(batch, torch.float32, flags=C.CQL_FLAG_DEBUG_SKIP_X)
     assert case.layer.device_status(batch) == C.CQL_ERR_TIMEOUT
+    ws, nbytes = case.layer.workspace(batch)
+    C.cql_workspace_init(ws, nbytes)                 # the rule after any device error
     y = case.forward(batch, torch.float32)
     assert case.layer.device_status(batch) == C.CQL_OK
     check_close(y, case.reference(batch), "f32", what=f"after timeout B={batch}")
