@@ -150,6 +150,7 @@ bool make_map_rowblocks(CUtensorMap* m, const void* plane, uint64_t block_bytes,
 
 // Prefill scratch (inside the forward workspace): byte offsets.
 struct PrefillLayout {
+  bool sparse;     // 2:4 int4: the sparse GEMM (weights dequantised on chip)
   int r3;          // adapter extension columns (3 r rounded up to 64)
   int rrows;       // R rows padded to 128
   int r_pad;       // rank rounded up to 32
@@ -159,5 +160,9 @@ struct PrefillLayout {
 PrefillLayout prefill_layout(const cql_desc& d, int m);
 bool prefill_supported(const cql_desc& d, int x_dt);
 cudaError_t launch_prefill(const DecodeParams& p, uint8_t* prefill_ws, cudaStream_t st);
+// The sparse-tensor-core GEMM of 2:4 int4 layers (prefill_sp.cu): lbuf holds
+// the adapter columns [N][r3], t3 the split T = X R^T [m][r3].
+cudaError_t launch_pf_sgemm(const DecodeParams& p, const uint16_t* lbuf, int r3, const uint16_t* t3, bool lowrank,
+                            cudaStream_t st);
 
 }  // namespace cql

@@ -16,12 +16,14 @@
 // "Low-rank adapter quantization"; the adapters are AbsMax int4 g128).
 //
 // Kernels, in stream order:
-//   k_pf_dequant   packed planes -> q as bf16 (2:4 expanded, zeros where
-//                  pruned) [N][K + r3], fp32 scales [N][K/128], and the same
-//                  for R (rows padded to 128); L^ hi/lo in the extra columns.
+//   k_pf_dequant_* R (rows padded to 128) as bf16 codes; L^ hi/lo as the
+//                  adapter columns; for the layers the sparse GEMM does not
+//                  take (int3, no mask) also q as bf16 (zeros where pruned)
+//                  [N][K + r3] and fp32 scales [N][K/128]
 //   k_pf_gemm      T-pass: T = X R^T (split over K, fp32 atomics)
 //   k_pf_tsplit    T -> [Thi | Tlo | Thi] bf16, clears the accumulator
-//   k_pf_gemm      main pass: Y = ...
+//   main pass      2:4 int4 layers: k_pf_sgemm (prefill_sp.cu, sparse tensor
+//                  cores, weights dequantised on chip); others: k_pf_gemm
 // Roles inside k_pf_gemm (one CTA per SM, persistent over 128x256 tiles):
 //   warp 0        TMA producer (4-stage ring of A 128x64 and B 256x64 tiles)
 //   warp 1        tensor-memory allocator and single-thread MMA issuer
@@ -251,52 +253,8 @@ CQL_DEV uint16_t to16(float v, int f16) { return f16 ? __half_as_ushort(__float2
 CQL_DEV float from16(uint16_t b, int f16) { return f16 ? f16_bits_to_f32(b) : bf16_bits_to_f32(b); }
 CQL_DEV uint16_t int_to16(int q, int f16) { return to16((float)q, f16); }   // exact for |q| <= 256
 
-// 2:4 int4 -> 16-bit codes, zeros where pruned.  A warp per (row block,
-// 128-column unit): coalesced 16-byte loads of its code and pattern slabs
-// (lane = row), branch-free expansion of each group (its META code holds the
-// kept positions i0 | i1 << 2), a transpose through
-// shared memory, then full-row 16-byte stores (two rows per instruction).
-constexpr int kDqWarps = 4;
-__global__ void __launch_bounds__(kDqWarps * 32) k_pf_dequant_w24(DecodeParams p, uint16_t* qbf, int ldq,
-                                                                  float* scales, int f16) {
-  __shared__ uint4 stage[kDqWarps][32][17];          // 17: pad against bank conflicts
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int G = p.upr;
-  const uint64_t wid = (uint64_t)blockIdx.x * kDqWarps + warp;
-  if (wid >= (uint64_t)p.n_rb * G) return;
-  const int rb = (int)(wid / G), g = (int)(wid % G);
-  const uint4 va = ldg_stream(p.values + slab_off(rb, 2 * g, p.rb.values) + lane * 16);
-  const uint4 vb = ldg_stream(p.values + slab_off(rb, 2 * g + 1, p.rb.values) + lane * 16);
-  const uint4 mm = ldg_stream(p.meta + slab_off(rb, g, p.rb.meta) + lane * 16);
-  const uint32_t sc16 = ldg_u16(p.scales + rit((uint64_t)rb * 32 + lane, 2 * g, p.rb.scales));
-  const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-  const uint32_t mw[4] = {mm.x, mm.y, mm.z, mm.w};
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {                     // 8 columns = 2 groups per 16-byte chunk
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int gi = 2 * c + h;
-      const uint32_t pt = (mw[gi >> 3] >> (4 * (gi & 7))) & 15u;
-      const uint32_t i0 = pt & 3u, i1 = pt >> 2;
-      const uint32_t byte = (vw[gi >> 2] >> (8 * (gi & 3))) & 0xFFu;
-      const uint32_t q0 = int_to16((int)(byte & 15u) - 8, f16), q1 = int_to16((int)(byte >> 4) - 8, f16);
-      w[2 * h] = (i0 == 0 ? q0 : 0u) | ((i0 == 1 ? q0 : (i1 == 1 ? q1 : 0u)) << 16);
-      w[2 * h + 1] = (i0 == 2 ? q0 : (i1 == 2 ? q1 : 0u)) | ((i1 == 3 ? q1 : 0u) << 16);
-    }
-    stage[warp][lane][c] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  __syncwarp();
-  const int half = lane >> 4, c = lane & 15;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int row = 2 * i + half;
-    *reinterpret_cast<uint4*>(qbf + (uint64_t)(rb * 32 + row) * ldq + (uint64_t)g * 128 + c * 8) = stage[warp][row][c];
-  }
-  scales[(uint64_t)(rb * 32 + lane) * G + g] = f16_bits_to_f32(sc16);
-}
-
-// Any uniform codec with the 2:4 mask or no mask (generic bit extraction).
+// Codes of the layers the sparse GEMM does not take (int3 2:4, no mask) as
+// 16-bit integers, zeros where pruned (generic bit extraction).
 __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* scales, int f16) {
   const int G = p.upr;
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -352,9 +310,11 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
 }
 
 // Adapter columns of the main operand: [Lhi | Lhi | Llo | 0] at columns
-// K .. K + r3 of row n, with L^ = q_L s_L exact in fp32 and Lhi + Llo = L^.
+// col0 .. col0 + r3 of row n, with L^ = q_L s_L exact in fp32 and
+// Lhi + Llo = L^ (col0 = K after the dense codes; 0 in the separate adapter
+// buffer of the sparse GEMM).
 // A thread per (row, 8 columns): one 16-byte store.
-__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3, int f16) {
+__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int col0, int r3, int f16) {
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int r = p.d.rank, chunks = r3 / 8;
   if (id >= (uint64_t)p.d.n_out * chunks) return;
@@ -375,7 +335,7 @@ __global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int r3, i
     }
     w[i >> 1] |= v << (16 * (i & 1));
   }
-  *reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + p.d.k_in + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + col0 + c0) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // R rows (padded to 128) as bf16 codes and fp32 scales.
@@ -420,10 +380,13 @@ PrefillLayout prefill_layout(const cql_desc& d, int m) {
   L.r3 = r ? (int)((3 * r + 63) / 64 * 64) : 0;
   L.rrows = r ? (int)((r + 127) / 128 * 128) : 0;
   L.r_pad = (int)((r + 31) / 32 * 32);
-  L.ldq = (int)(k + L.r3);
+  L.sparse = d.mask == CQL_MASK_2_4 && d.codec == CQL_CODEC_INT4_SYM;
+  // the sparse GEMM dequantises the weights on chip: only the adapter
+  // columns [N][r3] are staged in memory
+  L.ldq = L.sparse ? L.r3 : (int)(k + L.r3);
   uint64_t pos = 0;
   L.qbf = pos;     pos = align256(pos + n * L.ldq * 2);
-  L.wsc = pos;     pos = align256(pos + n * (k / 128) * 4);
+  L.wsc = pos;     pos = align256(pos + (L.sparse ? 0 : n * (k / 128) * 4));
   L.rbf = pos;     pos = align256(pos + (uint64_t)L.rrows * k * 2);
   L.rsc = pos;     pos = align256(pos + (uint64_t)L.rrows * (k / 128) * 4);
   L.tacc = pos;    pos = align256(pos + (uint64_t)m * L.r_pad * 4);
@@ -477,15 +440,13 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   const size_t smem = sizeof(PfSmem) + 1024;
   if ((e = ensure_smem_attr(attr_done, (const void*)k_pf_gemm, (int)smem)) != cudaSuccess) return e;
   const uint64_t nw = (uint64_t)N * G;
-  if (p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM)
-    k_pf_dequant_w24<<<(unsigned)(((uint64_t)p.n_rb * G + kDqWarps - 1) / kDqWarps), kDqWarps * 32, 0, st>>>(
-        p, qbf, L.ldq, wsc, f16);
-  else
+  if (!L.sparse) {
     k_pf_dequant_w<<<(unsigned)((nw + 127) / 128), 128, 0, st>>>(p, qbf, L.ldq, wsc, f16);
-  if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);       // main term off: zero scales
+    if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);     // main term off: zero scales
+  }
   if (lowrank) {
     const uint64_t nl = (uint64_t)N * (L.r3 / 8);
-    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.r3, f16);
+    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.sparse ? 0 : K, L.r3, f16);
     const uint64_t nr = (uint64_t)L.rrows * K;
     k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows, f16);
   }
@@ -513,6 +474,7 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
   } else {
     mT = mB;
   }
+  if (L.sparse) return launch_pf_sgemm(p, qbf, L.r3, t3, lowrank, st);
   if (!make_map(&mA, qbf, (uint64_t)N, (uint64_t)L.ldq, (uint64_t)L.ldq, PF_BM)) return cudaErrorInvalidValue;
   PfGemmParams g{};
   g.scales = wsc; g.rows = N; g.m = m; g.groups = G; g.lr_blocks = lowrank ? L.r3 / PF_BK : 0;
