@@ -17,6 +17,11 @@ Sources (web pages summarising the methods):
 * SqueezeLLM: Dense-and-Sparse Quantization -- "Approach" (non-uniform LUT
   quantisation; the top 0.45% outliers go to a full-precision CSR matrix so
   the dense part has a narrower range).
+* SLiM (same page), rebuttal "Output Error Minimization in SLiM-Quant": the
+  output-error variant scales the weights of the ~1% most salient input
+  channels up by a factor and the matching activations down by it; a
+  channel's saliency is the product of the normalised mean magnitudes of its
+  activations and of its weights.
 
 Where the pages are silent the plainest reading is taken; every such reading
 is listed in the design notes and repeated at the function that makes it.
@@ -49,10 +54,12 @@ __all__ = [
     "quantize_uniform", "lut_centroids", "lut_assign",
     "quantize_adapter_rows", "quantize_adapter_cols",
     "build_csr", "compress", "packed_layout", "pack_bytes",
+    "channel_saliency", "select_salient_channels", "scale_activations",
     "forward", "forward_terms", "dense_reconstruction",
     "rel_err", "pack_and_forward", "HEADER_BYTES", "NPLANES",
     "P_HEADER", "P_VALUES", "P_META", "P_SCALES", "P_VOFF", "P_CSR_ROWPTR",
     "P_CSR_COL", "P_CSR_VAL", "P_R_VALUES", "P_R_SCALES", "P_L_VALUES", "P_L_SCALES",
+    "P_SALIENT", "FORMAT_VERSION",
 ]
 
 # ---------------------------------------------------------------------------
@@ -88,6 +95,8 @@ class OracleDesc:
     adapter_bits: int = 4
     adapter_group: int = GROUP
     flags: int = 0
+    salient_channels: int = 0   # SLiM^O: channels scaled (0 = plain SLiM)
+    salient_log2: int = 0       # SLiM^O: the factor is 2**salient_log2
 
 
 def desc_for(wl) -> OracleDesc:
@@ -95,7 +104,9 @@ def desc_for(wl) -> OracleDesc:
     mask = {"2:4": MASK_2_4, "bitmap50": MASK_BITMAP50, "none": MASK_NONE}[wl.mask]
     codec = {"int4": CODEC_INT4, "int3": CODEC_INT3, "lut3": CODEC_LUT3,
              "lut4": CODEC_LUT4}[wl.codec]
-    return OracleDesc(wl.n, wl.k, mask, codec, wl.clip_alpha, wl.outlier_frac, wl.rank)
+    return OracleDesc(wl.n, wl.k, mask, codec, wl.clip_alpha, wl.outlier_frac, wl.rank,
+                      salient_channels=getattr(wl, "salient_channels", 0),
+                      salient_log2=getattr(wl, "salient_log2", 0))
 
 
 def _f32(v: float) -> float:
@@ -328,12 +339,75 @@ def build_csr(w: np.ndarray, out_idx: np.ndarray, dense_val: np.ndarray):
 
 
 # ---------------------------------------------------------------------------
+# salient-channel scaling (SLiM rebuttal, "Output Error Minimization in
+# SLiM-Quant"; the variant is called SLiM^O there)
+# ---------------------------------------------------------------------------
+
+SALIENT_ROW_BLOCK = 64      # rows per partial sum of a channel's |w|
+
+
+def channel_saliency(w: np.ndarray, act_absmean: np.ndarray) -> np.ndarray:
+    """Saliency of every input channel c: mean|x_c| * sum_n |w[n, c]|, fp64.
+
+    The page defines it as the product of the normalised average magnitudes
+    of the channel's activations and weights.  Dividing either factor by a
+    positive constant (its mean, its maximum, or N for the weight average)
+    does not change which channels rank highest, so the plain product of the
+    activation statistic and the column's |w| sum is kept (reading).  The
+    activation statistic is an input (measured on calibration data by the
+    caller; synthetic here), taken as float32 and widened exactly.
+
+    Summation order (fixed so that an implementation can reproduce the fp64
+    result bit for bit): rows in consecutive blocks of 64, each block summed
+    from its first row on, then the block sums added from the first block
+    on."""
+    w = np.abs(np.asarray(w, dtype=np.float64))
+    n, k = w.shape
+    assert n % SALIENT_ROW_BLOCK == 0
+    nb = n // SALIENT_ROW_BLOCK
+    blocks = w.reshape(nb, SALIENT_ROW_BLOCK, k)
+    part = np.zeros((nb, k))
+    for i in range(SALIENT_ROW_BLOCK):
+        part += blocks[:, i, :]
+    colsum = np.zeros(k)
+    for b in range(nb):
+        colsum += part[b]
+    a = np.asarray(act_absmean, dtype=np.float32).astype(np.float64)
+    assert a.shape == (k,)
+    return a * colsum
+
+
+def select_salient_channels(w: np.ndarray, act_absmean: np.ndarray, count: int) -> np.ndarray:
+    """Ascending indices of the ``count`` channels of highest saliency (ties
+    to the lower channel index; reading: the page names no tie rule)."""
+    sal = channel_saliency(w, act_absmean)
+    order = np.lexsort((np.arange(sal.size), -sal))   # saliency descending, then index
+    return np.sort(order[:count]).astype(np.int64)
+
+
+def scale_activations(x: np.ndarray, salient: np.ndarray, log2: int) -> np.ndarray:
+    """x with the salient channels divided by the factor 2**log2 (the inverse
+    of the weights' scaling; exact in fp64)."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    x[:, salient] = x[:, salient] / float(2 ** log2)
+    return x
+
+
+# ---------------------------------------------------------------------------
 # the whole encoding
 # ---------------------------------------------------------------------------
 
 def compress(desc: OracleDesc, w: np.ndarray, L: Optional[np.ndarray] = None,
-             R: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
-    """Run the encoding steps in order: outliers, mask, codec, CSR, adapters.
+             R: Optional[np.ndarray] = None, act_absmean: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """Run the encoding steps in order: (SLiM^O) salient-channel scaling,
+    outliers, mask, codec, CSR, adapters.
+
+    With ``desc.salient_channels`` > 0 the chosen columns of W are multiplied
+    by 2**salient_log2 before every other step, which then all work on the
+    scaled matrix W'; the forward pass divides the same activation channels
+    by the factor, so W' x' = W x before compression.  (Reading: the page
+    leaves the factor's value unstated; a power of two keeps both scalings
+    exact.  The adapters L, R are taken as given, acting on x'.)
 
     Returns the decoded parts the forward pass needs plus the raw codes the
     packer serialises."""
@@ -341,6 +415,13 @@ def compress(desc: OracleDesc, w: np.ndarray, L: Optional[np.ndarray] = None,
     n, k = w.shape
     assert (n, k) == (desc.n_out, desc.k_in)
     parts: Dict[str, np.ndarray] = {}
+    if desc.salient_channels > 0:
+        assert act_absmean is not None and desc.salient_log2 > 0
+        sal = select_salient_channels(w, act_absmean, desc.salient_channels)
+        w = w.copy()
+        w[:, sal] = w[:, sal] * float(2 ** desc.salient_log2)
+        parts["salient"] = sal
+        parts["salient_log2"] = np.int64(desc.salient_log2)
     ns = n_outliers(desc)
     out_idx = select_outliers(w, ns)
     is_out = np.zeros(n * k, dtype=bool)
@@ -396,8 +477,11 @@ def forward_terms(parts: Dict[str, np.ndarray], x: np.ndarray, rows=None):
 
     ``rows`` optionally restricts the output to a subset of output rows (used
     for sampled parity at full size).  Returns (main, csr, lowrank), each
-    [B][len(rows)]."""
+    [B][len(rows)].  A SLiM^O layer first divides its salient activation
+    channels by the factor."""
     x = np.asarray(x, dtype=np.float64)
+    if "salient" in parts:
+        x = scale_activations(x, parts["salient"], int(parts["salient_log2"]))
     wd = parts["w_dense"]
     sel = np.arange(wd.shape[0]) if rows is None else np.asarray(rows)
     main = x @ wd[sel].T
@@ -430,7 +514,9 @@ def forward(parts: Dict[str, np.ndarray], x: np.ndarray, rows=None, flags: int =
 
 
 def dense_reconstruction(parts: Dict[str, np.ndarray]) -> np.ndarray:
-    """W_hat = deq(Q (.) M) + S + deq(L) deq(R) as one dense fp64 matrix."""
+    """W_hat = deq(Q (.) M) + S + deq(L) deq(R) as one dense fp64 matrix, in
+    the original channel scale (a SLiM^O layer's salient columns divided by
+    the factor), so that forward(x) = x W_hat^T."""
     wd = parts["w_dense"].copy()
     if "csr_row_ptr" in parts:
         rp, col, val = parts["csr_row_ptr"], parts["csr_col"], parts["csr_val"]
@@ -438,6 +524,9 @@ def dense_reconstruction(parts: Dict[str, np.ndarray]) -> np.ndarray:
         np.add.at(wd, (rows, col), val)
     if "R_hat" in parts:
         wd = wd + parts["L_hat"] @ parts["R_hat"]
+    if "salient" in parts:
+        sal = parts["salient"]
+        wd[:, sal] = wd[:, sal] / float(2 ** int(parts["salient_log2"]))
     return wd
 
 
@@ -458,9 +547,10 @@ def rel_err(y: np.ndarray, ref: np.ndarray) -> float:
 # ---------------------------------------------------------------------------
 
 HEADER_BYTES = 512
-NPLANES = 12
+FORMAT_VERSION = 2
+NPLANES = 13
 (P_HEADER, P_VALUES, P_META, P_SCALES, P_VOFF, P_CSR_ROWPTR, P_CSR_COL,
- P_CSR_VAL, P_R_VALUES, P_R_SCALES, P_L_VALUES, P_L_SCALES) = range(NPLANES)
+ P_CSR_VAL, P_R_VALUES, P_R_SCALES, P_L_VALUES, P_L_SCALES, P_SALIENT) = range(NPLANES)
 
 
 def _pad16(x: int) -> int:
@@ -515,6 +605,7 @@ def packed_layout(desc: OracleDesc, nnz: Optional[int] = None) -> dict:
         ln[P_R_SCALES] = rpad * rb[P_R_SCALES]
         ln[P_L_VALUES] = n * rb[P_L_VALUES]
         ln[P_L_SCALES] = 2 * (n // GROUP) * r
+    ln[P_SALIENT] = 2 * desc.salient_channels
     off = [0] * NPLANES
     pos = 0
     for i in range(NPLANES):
@@ -560,14 +651,14 @@ def _f16_bits(v: np.ndarray) -> np.ndarray:
 
 def _header(desc: OracleDesc, lay: dict) -> np.ndarray:
     d = struct.pack(
-        "<iiiiiffiiiI20x",
+        "<iiiiiffiiiIii12x",
         desc.n_out, desc.k_in, desc.mask, desc.codec, desc.group,
         np.float32(desc.clip_alpha), np.float32(desc.outlier_frac), desc.rank,
-        desc.adapter_bits, desc.adapter_group, desc.flags)
+        desc.adapter_bits, desc.adapter_group, desc.flags, desc.salient_channels, desc.salient_log2)
     assert len(d) == 64
-    body = b"CQL1" + struct.pack("<I", 1) + d
+    body = b"CQL1" + struct.pack("<I", FORMAT_VERSION) + d
     body += struct.pack("<QQ", lay["total"], lay["nnz"])
-    body += struct.pack("<12Q", *lay["off"]) + struct.pack("<12Q", *lay["len"])
+    body += struct.pack(f"<{NPLANES}Q", *lay["off"]) + struct.pack(f"<{NPLANES}Q", *lay["len"])
     out = np.zeros(HEADER_BYTES, dtype=np.uint8)
     out[: len(body)] = np.frombuffer(body, dtype=np.uint8)
     return out
@@ -634,10 +725,12 @@ def pack_bytes(desc: OracleDesc, parts: Dict[str, np.ndarray]) -> np.ndarray:
         lc = (parts["L_q"].astype(np.int16) + 8).astype(np.uint8)
         put(P_L_VALUES, _interleave(_bitstream(lc, 4, rb[P_L_VALUES])))
         put(P_L_SCALES, _u16le(_f16_bits(parts["L_s"])).reshape(-1))
+    if desc.salient_channels > 0:
+        put(P_SALIENT, _u16le(parts["salient"].astype(np.uint16)))
     return buf
 
 
-def pack_and_forward(desc: OracleDesc, w, L, R, x):
+def pack_and_forward(desc: OracleDesc, w, L, R, x, act_absmean=None):
     """Convenience: (packed bytes, parts, y fp64)."""
-    parts = compress(desc, w, L, R)
+    parts = compress(desc, w, L, R, act_absmean)
     return pack_bytes(desc, parts), parts, forward(parts, x)

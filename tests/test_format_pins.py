@@ -44,11 +44,12 @@ def f16(bits):
 def parse_header(buf):
     assert bytes(buf[:4]) == b"CQL1"
     (ver,) = struct.unpack_from("<I", bytes(buf[:8]), 4)
-    d = struct.unpack_from("<iiiiiffiiiI", bytes(buf[:72]), 8)
+    d = struct.unpack_from("<iiiiiffiiiIii", bytes(buf[:72]), 8)
+    assert not any(buf[60:72])                      # reserved descriptor words
     total, nnz = struct.unpack_from("<QQ", bytes(buf[:88]), 72)
-    off = struct.unpack_from("<12Q", bytes(buf[:280]), 88)
-    ln = struct.unpack_from("<12Q", bytes(buf[:280]), 184)
-    assert not any(buf[280:512])
+    off = struct.unpack_from("<13Q", bytes(buf[:296]), 88)
+    ln = struct.unpack_from("<13Q", bytes(buf[:296]), 192)
+    assert not any(buf[296:512])
     return ver, d, total, nnz, list(off), list(ln)
 
 
@@ -59,6 +60,8 @@ CASES = [
     ("down_unstructured", dict(n=128, k=384, rank=16)),
     ("lut_dense_sparse", dict(n=128, k=256)),
     ("lut_dense_sparse", dict(n=128, k=256, codec="lut4")),
+    ("mlp_up_slimo", dict(n=128, k=512, rank=16, salient_channels=5, salient_log2=1)),
+    ("lut_dense_sparse", dict(n=128, k=256, salient_channels=32, salient_log2=3)),
 ]
 
 
@@ -67,16 +70,23 @@ def test_packed_bytes_decode_to_parts(name, over):
     wl = workload(name, **over)
     inp = make_layer_inputs(wl, max_batch=1)
     d = O.desc_for(wl)
-    parts = O.compress(d, inp["w"], inp["L"], inp["R"])
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
     buf = O.pack_bytes(d, parts)
     ver, hd, total, nnz, off, ln = parse_header(buf)
-    assert ver == 1 and total == buf.size
+    assert ver == 2 and total == buf.size
     assert hd[:5] == (d.n_out, d.k_in, d.mask, d.codec, 128) and hd[7] == d.rank
+    assert hd[11:13] == (d.salient_channels, d.salient_log2)
     n, k, r = d.n_out, d.k_in, d.rank
     bits = {0: 4, 1: 3, 2: 3, 3: 4}[d.codec]
     plane = lambda p: buf[off[p]: off[p] + ln[p]]
-    for p in range(12):
+    for p in range(13):
         assert off[p] % 256 == 0
+    if d.salient_channels:
+        sal = np.frombuffer(bytes(plane(O.P_SALIENT)), dtype="<u2")
+        assert len(sal) == d.salient_channels and (np.diff(sal.astype(int)) > 0).all()
+        assert (sal == parts["salient"]).all()
+    else:
+        assert ln[O.P_SALIENT] == 0
     keep = parts["keep"]
 
     vals = plane(O.P_VALUES)

@@ -469,3 +469,136 @@ def test_rel_err_metric():
     rms = math.sqrt((1 + 4 + 0 + 1e-18) / 4)
     y = ref + np.array([[0.0, 0.004, 1e-3, 0.0]])
     assert abs(O.rel_err(y, ref) - max(0.004 / 2.0, 1e-3 / rms)) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# SLiM^O salient-channel scaling (SLiM rebuttal, "Output Error Minimization
+# in SLiM-Quant")
+# ---------------------------------------------------------------------------
+
+def _brute_salient(w, act, m):
+    """Exact rational saliency (mean|x_c| * sum_n |w_nc|) and the m channels
+    that rank first (saliency descending, lower index on ties), pure Python."""
+    n, k = w.shape
+    sal = []
+    for c in range(k):
+        s = sum(Fraction(abs(float(w[i, c]))) for i in range(n))
+        sal.append(Fraction(float(np.float32(act[c]))) * s)
+    order = sorted(range(k), key=lambda c: (-sal[c], c))
+    return sorted(order[:m])
+
+
+def test_salient_selection_brute_force_with_ties():
+    """Dyadic weights and statistics make every fp64 sum exact, so the
+    oracle's ranking must equal the exact one.  Channels 3 and 9 tie exactly
+    (half the |w| sum, twice the statistic) and sit at the cut: four channels
+    rank above them, so the fifth pick must be the lower index, 3."""
+    rng = np.random.default_rng(7)
+    n, k, m = 128, 16, 5
+    mag = np.array([(c % 5 + 1) / 64.0 for c in range(k)])
+    mag[3], mag[9] = 4 / 64.0, 2 / 64.0
+    w = mag[None, :] * rng.choice([-1.0, 1.0], size=(n, k))
+    act = (np.arange(k) + 1) / 4.0
+    others = sorted((act[c] * n * mag[c] for c in range(k) if c not in (3, 9)), reverse=True)
+    v = math.floor((others[3] + others[4]) / 2 * 8) / 8      # dyadic, strictly between 4th and 5th
+    assert others[4] < v < others[3]
+    act[3], act[9] = v / (n * mag[3]), 2 * v / (n * mag[3])
+    got = list(O.select_salient_channels(w, act, m))
+    assert got == _brute_salient(w, act, m)
+    assert 3 in got and 9 not in got
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_salient_selection_brute_force_random(seed):
+    rng = np.random.default_rng(100 + seed)
+    n, k, m = 64, 40, 7
+    w = rng.standard_normal((n, k)) * 0.02
+    act = np.exp(0.5 * rng.standard_normal(k)).astype(np.float32)
+    assert list(O.select_salient_channels(w, act, m)) == _brute_salient(w, act, m)
+
+
+def test_saliency_normalisation_does_not_change_the_choice():
+    """The page multiplies the *normalised* mean magnitudes of activations
+    and weights; dividing each factor by its mean (or maximum) and the weight
+    sum by N leaves the selected set unchanged."""
+    rng = np.random.default_rng(11)
+    n, k, m = 256, 512, 5
+    w = rng.standard_normal((n, k)) * 0.02
+    act = np.exp(0.5 * rng.standard_normal(k)).astype(np.float32)
+    a = act.astype(np.float64)
+    wbar = np.abs(w).mean(axis=0)
+    for na, nw in ((a.mean(), wbar.mean()), (a.max(), wbar.max())):
+        s = (a / na) * (wbar / nw)
+        top = np.sort(np.argsort(-s, kind="stable")[:m])
+        assert (top == O.select_salient_channels(w, act, m)).all()
+
+
+def test_slimo_is_plain_compression_of_the_scaled_matrix():
+    """Wiring: a SLiM^O layer equals the plain pipeline run on W with the
+    chosen columns doubled (scaled here, independently), and its forward
+    equals the plain forward on x with those channels halved -- bit for bit."""
+    wl = workload("mlp_up_slimo", n=256, k=512, rank=16, salient_channels=6, salient_log2=1)
+    inp = make_layer_inputs(wl, max_batch=3)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
+    sal = parts["salient"]
+    assert len(sal) == 6
+    w2 = inp["w"].astype(np.float64).copy()
+    for c in sal:
+        w2[:, c] *= 2.0
+    dp = O.OracleDesc(d.n_out, d.k_in, d.mask, d.codec, d.clip_alpha, d.outlier_frac, d.rank)
+    plain = O.compress(dp, w2, inp["L"], inp["R"])
+    for key in ("q", "scales", "keep", "R_q", "L_q"):
+        assert (parts[key] == plain[key]).all(), key
+    x = inp["x"].astype(np.float64)
+    x2 = x.copy()
+    for c in sal:
+        x2[:, c] /= 2.0
+    assert (O.forward(parts, x) == O.forward(plain, x2)).all()
+
+
+def test_slimo_lossless_grid_matrix_reproduces_wx_exactly():
+    """Closed form: W on the int4 grid (each group's maximum 7 s in a
+    non-salient column, salient columns at most 3 s) stays on the grid after
+    the salient columns are doubled, so with alpha = 1 and no mask the SLiM^O
+    layer reproduces W x exactly -- scaling W's channel by 2 and x's by 1/2
+    leaves y unchanged."""
+    rng = np.random.default_rng(5)
+    n, k = 128, 256
+    s = 2.0 ** -6
+    q = rng.integers(-7, 8, size=(n, k))
+    salient = [5, 130, 200]
+    q[:, salient] = rng.integers(-3, 4, size=(n, len(salient)))
+    q[:, 0] = 7
+    q[:, 128] = -7                                    # every group's max, non-salient
+    w = q * s
+    act = np.ones(k, dtype=np.float32)
+    act[salient] = 1000.0
+    d = O.OracleDesc(n, k, O.MASK_NONE, O.CODEC_INT4, clip_alpha=1.0, salient_channels=3, salient_log2=1)
+    parts = O.compress(d, w, act_absmean=act)
+    assert list(parts["salient"]) == salient
+    assert (parts["scales"] == s).all()
+    x = rng.integers(-8, 9, size=(4, k)) / 8.0
+    assert (O.forward(parts, x) == x @ w.T).all()
+    assert (O.dense_reconstruction(parts) == w).all()
+
+
+def test_slimo_reduces_the_error_of_the_salient_channels():
+    """The effect the page reports: with the salient columns scaled by 2 the
+    reconstruction error on those columns drops, on random Gaussian weights.
+    Not by half: a doubled entry sometimes sets its group's maximum (a coarser
+    step for the whole group) or lands above the alpha = 0.9 clip; about a
+    quarter less on this draw (0.76 of the plain error)."""
+    wl = workload("mlp_up_slimo", n=512, k=1024, rank=0, spike_frac=0.0, salient_channels=10, salient_log2=1)
+    inp = make_layer_inputs(wl, max_batch=1)
+    d = O.desc_for(wl)
+    dense = O.OracleDesc(d.n_out, d.k_in, O.MASK_NONE, d.codec, d.clip_alpha)
+    dense_s = O.OracleDesc(d.n_out, d.k_in, O.MASK_NONE, d.codec, d.clip_alpha, salient_channels=10,
+                           salient_log2=1)
+    w = inp["w"].astype(np.float64)
+    ps = O.compress(dense_s, w, act_absmean=inp["act_absmean"])
+    pp = O.compress(dense, w)
+    sal = ps["salient"]
+    err_s = np.abs(O.dense_reconstruction(ps)[:, sal] - w[:, sal]).mean()
+    err_p = np.abs(O.dense_reconstruction(pp)[:, sal] - w[:, sal]).mean()
+    assert err_s < 0.85 * err_p, (err_s, err_p)

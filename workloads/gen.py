@@ -10,7 +10,11 @@ the same value structure the workload descriptions ask for:
   split and SLiM's clipping are designed for);
 * Student-t(4) weights for the dense-and-sparse LUT workload (heavier tails);
 * rank-r adapter factors drawn as 0.01 N(0, 1);
-* activations drawn as N(0, 1).
+* activations drawn as N(0, 1);
+* for the output-error (SLiM^O) variant, a per-channel activation statistic
+  mean|x_c| drawn as exp(0.5 N(0, 1)) with 0.5% of the channels multiplied by
+  30 (the few "massive" activation channels LLMs show), from its own stream
+  (PCG64 seeded with (seed, 1)) so the other draws are unchanged.
 
 Every array is drawn from ``numpy.random.default_rng(seed)`` (PCG64) in a fixed
 order: W, the spike positions, L, R, x.  Nothing here masks, quantises or
@@ -85,6 +89,8 @@ class Workload:
     x_dtype: str = "bf16"       # "f16" or "bf16"
     batches: Tuple[int, ...] = (1,)
     note: str = ""
+    salient_channels: int = 0   # SLiM^O: channels scaled (0 = plain SLiM)
+    salient_log2: int = 0       # SLiM^O: factor 2**salient_log2
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -122,6 +128,13 @@ WORKLOADS: Dict[str, Workload] = {
         mask="2:4", codec="int4", clip_alpha=0.9, rank=64, x_dtype="bf16",
         batches=(2048,),
         note="2048 tokens x (4096 -> 11008); 2:4 int4 g128 + rank-64 adapters"),
+    # Output-error variant (SLiM^O) of the MLP up projection: the 1% most
+    # salient input channels (41 of 4096) scaled by 2.
+    "mlp_up_slimo": Workload(
+        name="mlp_up_slimo", seed=7, n=11008, k=4096, w_dtype="bf16",
+        spike_frac=0.001, mask="2:4", codec="int4", clip_alpha=0.9,
+        rank=128, x_dtype="bf16", batches=(1, 16), salient_channels=41, salient_log2=1,
+        note="mlp_up with SLiM^O: top 1% salient channels (41) x2, activations /2"),
     "prefill_down": Workload(
         name="prefill_down", seed=6, n=4096, k=11008, w_dtype="bf16",
         mask="2:4", codec="int4", clip_alpha=0.9, rank=64, x_dtype="bf16",
@@ -171,7 +184,9 @@ def make_layer_inputs(wl: Workload, max_batch: Optional[int] = None) -> dict:
       ``L``      float32 [N][r] (or None when rank == 0),
       ``R``      float32 [r][K] (or None),
       ``x``      float32 [B][K], the exact delivered activation values,
-      ``x_bits`` uint16 [B][K] (fp16 or bf16 patterns).
+      ``x_bits`` uint16 [B][K] (fp16 or bf16 patterns),
+      ``act_absmean`` float32 [K] per-channel mean |x| statistic (SLiM^O
+                 workloads; None otherwise).
     """
     rng = np.random.default_rng(wl.seed)
     n, k = wl.n, wl.k
@@ -192,7 +207,14 @@ def make_layer_inputs(wl: Workload, max_batch: Optional[int] = None) -> dict:
         R = (rng.standard_normal((wl.rank, k)) * wl.lr_std).astype(np.float32)
     bmax = max_batch if max_batch is not None else max(wl.batches)
     x32, x_bits = _deliver(rng.standard_normal((bmax, k)), wl.x_dtype)
-    return {"w": w32, "w_bits": w_bits, "L": L, "R": R, "x": x32, "x_bits": x_bits}
+    act = None
+    if wl.salient_channels > 0:
+        arng = np.random.default_rng((wl.seed, 1))
+        a = np.exp(0.5 * arng.standard_normal(k))
+        heavy = arng.choice(k, size=max(1, k // 200), replace=False)
+        a[heavy] *= 30.0
+        act = a.astype(np.float32)
+    return {"w": w32, "w_bits": w_bits, "L": L, "R": R, "x": x32, "x_bits": x_bits, "act_absmean": act}
 
 
 def make_activations(k: int, batch: int, dtype: str, seed: int):
