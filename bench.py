@@ -82,7 +82,7 @@ PLANE_HEADER, PLANE_VOFF = 0, 4          # include/cql.h CQL_PLANE_HEADER / CQL_
 def algorithmic_bytes(layout, batch, n, k, x_bytes=2, y_bytes=2):
     """Bytes the layer must move per call: every packed plane except the header
     and the VOFF index (a format aid), plus x and y."""
-    planes = sum(int(layout.len[i]) for i in range(12) if i not in (PLANE_HEADER, PLANE_VOFF))
+    planes = sum(int(layout.len[i]) for i in range(len(layout.len)) if i not in (PLANE_HEADER, PLANE_VOFF))
     return planes + batch * k * x_bytes + batch * n * y_bytes
 
 
@@ -90,7 +90,7 @@ def algorithmic_bytes_oracle(O, wl, batch):
     """The same byte count from the oracle's copy of the packed layout (the
     reference arm touches no GPU)."""
     lay = O.packed_layout(O.desc_for(wl))
-    planes = sum(int(lay["len"][i]) for i in range(12) if i not in (PLANE_HEADER, PLANE_VOFF))
+    planes = sum(int(lay["len"][i]) for i in range(len(lay["len"])) if i not in (PLANE_HEADER, PLANE_VOFF))
     return planes + batch * wl.k * 2 + batch * wl.n * 2
 
 
@@ -98,7 +98,8 @@ def desc_from_workload(C, wl):
     mask = {"2:4": C.CQL_MASK_2_4, "bitmap50": C.CQL_MASK_BITMAP50, "none": C.CQL_MASK_NONE}[wl.mask]
     codec = {"int4": C.CQL_CODEC_INT4_SYM, "int3": C.CQL_CODEC_INT3_SYM, "lut3": C.CQL_CODEC_LUT3_ROW,
              "lut4": C.CQL_CODEC_LUT4_ROW}[wl.codec]
-    return C.make_desc(wl.n, wl.k, mask, codec, wl.clip_alpha, wl.outlier_frac, wl.rank)
+    return C.make_desc(wl.n, wl.k, mask, codec, wl.clip_alpha, wl.outlier_frac, wl.rank, 0,
+                       wl.salient_channels, wl.salient_log2)
 
 
 def device_inputs(torch, inp, wl, dev):
@@ -117,10 +118,12 @@ def device_inputs(torch, inp, wl, dev):
 def kernels_per_step(wl, batch):
     """Kernels one decode call launches: the tensor-core path (2:4 int4) runs
     the main kernel (which also adds the CSR rows and R x) and the epilogue;
-    the CUDA-core paths add a pre-kernel when there are adapters or outliers."""
+    the CUDA-core paths add a pre-kernel when there are adapters or outliers;
+    a SLiM^O layer adds the activation-scaling prologue."""
+    pro = 1 if wl.salient_channels else 0
     if wl.mask == "2:4" and wl.codec == "int4":
-        return 2
-    return 2 + (1 if (wl.rank or wl.outlier_frac) else 0)
+        return 2 + pro
+    return 2 + pro + (1 if (wl.rank or wl.outlier_frac) else 0)
 
 
 def source_hash():
@@ -205,10 +208,10 @@ def cpu_oracle_rate(wl, batch, seconds, steps=None, warmup=0):
     from workloads import make_layer_inputs
     inp = make_layer_inputs(wl, max_batch=batch)
     od = O.desc_for(wl)
-    parts = O.compress(od, inp["w"], inp["L"], inp["R"])
+    parts = O.compress(od, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
     lay = O.packed_layout(od)
     x = inp["x"][:batch].astype(np.float64)
-    planes = sum(lay["len"][i] for i in range(12) if i not in (O.P_HEADER, O.P_VOFF))
+    planes = sum(lay["len"][i] for i in range(len(lay["len"])) if i not in (O.P_HEADER, O.P_VOFF))
     per_row = planes / wl.n
     t0 = time.perf_counter()
     O.forward(parts, x, rows=np.arange(min(wl.n, 256)))
@@ -268,6 +271,7 @@ def bench_config(wl, batch, world):
 def wl_name(wl, batch):
     return (f"{wl.name} {wl.n}x{wl.k} {wl.mask} {wl.codec} g128"
             + (f" r{wl.rank}" if wl.rank else "") + (f" csr{wl.outlier_frac}" if wl.outlier_frac else "")
+            + (f" salient{wl.salient_channels}x{2 ** wl.salient_log2}" if wl.salient_channels else "")
             + f" batch {batch}")
 
 
@@ -284,7 +288,8 @@ class Bench:
         inp = make_layer_inputs(wl, max_batch=batch)
         W, L, R, x = device_inputs(torch, inp, wl, dev)
         self.desc = desc_from_workload(C, wl)
-        self.layer = C.CompressedLinear(self.desc, W, L, R)
+        act = None if inp["act_absmean"] is None else torch.from_numpy(inp["act_absmean"]).to(dev)
+        self.layer = C.CompressedLinear(self.desc, W, L, R, act_absmean=act)
         self.desc.flags = flags                     # forward-only flags (the packed header keeps 0)
         del W, L, R
         torch.cuda.synchronize()
@@ -481,7 +486,8 @@ def extra_lines(torch, C, dev, stream, barrier):
     out = []
     peak, _ = measured_peaks()
     for name, batch in (("mlp_up", 1), ("tiny", 1), ("mlp_up", 4), ("mlp_up", 16), ("lut_dense_sparse", 1),
-                        ("lut_dense_sparse", 8), ("down_unstructured", 1), ("down_unstructured", 16)):
+                        ("lut_dense_sparse", 8), ("down_unstructured", 1), ("down_unstructured", 16),
+                        ("mlp_up_slimo", 1), ("mlp_up_slimo", 16)):
         wl = workload(name)
         b = Bench(wl, batch, dev, torch, C)
         total, per, _ = b.timed(20000, 200, stream)
@@ -516,7 +522,8 @@ def extra_lines(torch, C, dev, stream, barrier):
                     "TFLOP/s_dense_equiv": round(dense / per / 1e12, 1),
                     "frac_dense_equiv_of_measured_bf16": round(dense / per / 1e12 / tf_peak, 4),
                     "TFLOP/s_algorithmic": round(algo / per / 1e12, 1),
-                    "note": "whole step: dequant to bf16 codes, T = X R^T pass, main tcgen05 GEMM"})
+                    "note": "whole step: adapter dequant, T = X R^T pass, sparse tcgen05 GEMM "
+                            "(2:4 codes converted on chip)"})
         del b
         torch.cuda.empty_cache()
     return out

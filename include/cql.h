@@ -12,10 +12,17 @@
  * split), and L_q, R_q rank-r adapters quantised AbsMax int4 in groups of 128
  * (SLiM's "Low-rank adapter quantization").
  *
+ * Output-error variant (SLiM^O; SLiM rebuttal, "Output Error Minimization in
+ * SLiM-Quant"): a layer packed with desc.salient_channels = m > 0 stores the
+ * compression of W' = W diag(sigma), where sigma_c = 2^salient_log2 on the m
+ * input channels of highest saliency and 1 elsewhere, and computes the
+ * formula above on x' = x diag(1/sigma): the forward divides those m
+ * activation channels by the factor before anything else reads x.
+ *
  * Sources: "SLiM: One-shot Quantization and Sparsity with Low-rank
  * Approximation for LLM Weight Compression" (review summary: SLIM-Quant,
  * Low-rank adapter quantization; rebuttal: Unstructured vs. 2:4 Sparsity,
- * Speedup Comparison without LoRA) and "SqueezeLLM: Dense-and-Sparse
+ * Speedup Comparison without LoRA, Output Error Minimization in SLiM-Quant) and "SqueezeLLM: Dense-and-Sparse
  * Quantization" (Approach; Key results).  The pages fix no API, byte layout,
  * scale dtype, rounding or tie rule; those are defined here.
  *
@@ -34,15 +41,15 @@
  *     aborts or traps.
  *
  * ------------------------------------------------------------------------
- * PACKED FORMAT (version 1)
+ * PACKED FORMAT (version 2)
  * ------------------------------------------------------------------------
  * A packed weight is one contiguous device buffer: a 512-byte header followed
- * by up to 11 planes, in the order of the CQL_PLANE_* indices.  Every plane
+ * by up to 12 planes, in the order of the CQL_PLANE_* indices.  Every plane
  * starts on a 256-byte boundary; an absent plane has length 0 and the offset
  * where it would start.  All multi-byte fields are little-endian.
  *
- * Header: "CQL1", uint32 version = 1, cql_desc (64 bytes), then the
- * cql_layout (uint64 total_bytes, uint64 nnz, uint64 off[12], uint64 len[12]);
+ * Header: "CQL1", uint32 version = 2, cql_desc (64 bytes), then the
+ * cql_layout (uint64 total_bytes, uint64 nnz, uint64 off[13], uint64 len[13]);
  * the rest of the 512 bytes is zero.
  *
  * Row-interleaved planes (VALUES, META, SCALES, VOFF, R_VALUES, R_SCALES,
@@ -85,10 +92,18 @@
  * L_VALUES  int4 codes u = q + 8 of L [N][r]; row_bytes = pad16(r/2).
  * L_SCALES  fp16 [N/128][r], plain row-major: scale of column j over rows
  *           [128g, 128g+128) at index g*r + j.
+ * SALIENT   uint16 [m], m = salient_channels: the scaled input channels,
+ *           ascending.  Absent when m = 0.
  *
  * Encoding rules (shared by pack_compressed_weight and the CPU oracle; every
  * real-valued step is evaluated in fp64 from exact widenings, then rounded to
  * fp16 round-to-nearest-even, ties in selections go to the lower index):
+ *   0. SLiM^O (m > 0 only): saliency of channel c = a_c * sum_n |w[n][c]|,
+ *      a_c the caller's float32 mean |x_c| over calibration tokens and the
+ *      sum taken in fp64 over consecutive blocks of 64 rows (each block from
+ *      its first row on, then the block sums from the first block on); the
+ *      m channels of largest saliency have their column multiplied by
+ *      2^salient_log2 (exact), and every rule below applies to that W';
  *   1. outliers: the floor(f*N*K) entries of largest |w| over the whole matrix;
  *   2. mask on |w|: 2:4 keeps the two largest of every 4 columns; bitmap50
  *      keeps the K/2 largest of every row;
@@ -111,9 +126,9 @@
 extern "C" {
 #endif
 
-#define CQL_VERSION 1
+#define CQL_VERSION 2
 #define CQL_HEADER_BYTES 512
-#define CQL_NPLANES 12
+#define CQL_NPLANES 13
 #define CQL_GROUP 128
 #define CQL_MAX_DECODE_BATCH 16
 
@@ -137,7 +152,8 @@ typedef enum { CQL_DT_F32 = 0, CQL_DT_F16 = 1, CQL_DT_BF16 = 2 } cql_dtype;
 enum {
   CQL_PLANE_HEADER = 0, CQL_PLANE_VALUES = 1, CQL_PLANE_META = 2, CQL_PLANE_SCALES = 3,
   CQL_PLANE_VOFF = 4, CQL_PLANE_CSR_ROWPTR = 5, CQL_PLANE_CSR_COL = 6, CQL_PLANE_CSR_VAL = 7,
-  CQL_PLANE_R_VALUES = 8, CQL_PLANE_R_SCALES = 9, CQL_PLANE_L_VALUES = 10, CQL_PLANE_L_SCALES = 11
+  CQL_PLANE_R_VALUES = 8, CQL_PLANE_R_SCALES = 9, CQL_PLANE_L_VALUES = 10, CQL_PLANE_L_SCALES = 11,
+  CQL_PLANE_SALIENT = 12
 };
 
 /* Term toggles (cql_desc.flags, read by compressed_linear_forward only; used
@@ -169,7 +185,9 @@ typedef struct cql_desc {
   int32_t adapter_bits;   /* must be 4                                       */
   int32_t adapter_group;  /* must be 128                                     */
   uint32_t flags;         /* CQL_FLAG_* term toggles                         */
-  int32_t reserved[5];    /* zero                                            */
+  int32_t salient_channels; /* SLiM^O scaled channels m, 0 <= m <= K/8; 0 = off */
+  int32_t salient_log2;   /* SLiM^O factor 2^e, e in [1, 8] when m > 0, else 0 */
+  int32_t reserved[3];    /* zero                                            */
 } cql_desc;
 
 typedef struct cql_layout {
@@ -199,7 +217,11 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
  *   W         device, [N][K] row-major, w_dt = CQL_DT_F32 or CQL_DT_BF16,
  *             16-byte aligned.
  *   L         device fp32 [N][r] row-major, or NULL when rank == 0.
- *   R         device fp32 [r][K] row-major, or NULL when rank == 0.
+ *   R         device fp32 [r][K] row-major, or NULL when rank == 0.  (With
+ *             SLiM^O the adapters act on x', the scaled activations.)
+ *   act_absmean  device fp32 [K], the mean |x_c| of each input channel over
+ *             calibration tokens (finite, >= 0); required when
+ *             salient_channels > 0, ignored (may be NULL) otherwise.
  *   packed    device, >= cql_layout.total_bytes, 256-byte aligned; every byte
  *             of it is written.
  *   workspace device scratch of >= cql_pack_workspace_size bytes, 256-byte
@@ -207,7 +229,7 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
  * The result is bit-exact with the CPU oracle on every byte.  Inputs must be
  * finite. */
 cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt,
-                                  const float* L, const float* R, void* packed,
+                                  const float* L, const float* R, const float* act_absmean, void* packed,
                                   uint64_t packed_bytes, void* workspace, uint64_t ws_bytes,
                                   cql_stream_t stream);
 
@@ -234,6 +256,10 @@ cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t s
  *             aligned.
  *   y         device [batch][N], y_dt = CQL_DT_F32, F16 or BF16, 16-byte
  *             aligned; fp32 accumulation, one final round to y_dt.
+ *   A SLiM^O layer (salient_channels > 0) first runs a small kernel that
+ *   writes x' (x with the salient channels divided by 2^salient_log2,
+ *   rounded to x_dt, exact unless a value falls into x_dt's subnormal range)
+ *   into the workspace; every later step reads x'.
  *   batch     1..16 runs the decode path: sparse tcgen05 MMAs for 2:4 int4
  *             layers with fp16/bf16 x, a CUDA-core GEMV for the other codecs
  *             and masks; larger batches run the tcgen05 tensor-core prefill

@@ -29,7 +29,7 @@ CQL_DT_F32, CQL_DT_F16, CQL_DT_BF16 = 0, 1, 2
 CQL_FLAG_NO_MAIN, CQL_FLAG_NO_CSR, CQL_FLAG_NO_LOWRANK = 1, 2, 4
 CQL_FLAG_DEBUG_SKIP_X = 0x100
 CQL_FLAG_CUDA_CORE = 0x200
-CQL_NPLANES = 12
+CQL_NPLANES = 13
 CQL_MAX_DECODE_BATCH = 16
 
 EXPORTED = (
@@ -44,7 +44,8 @@ class cql_desc(ctypes.Structure):
         ("n_out", ctypes.c_int32), ("k_in", ctypes.c_int32), ("mask", ctypes.c_int32),
         ("codec", ctypes.c_int32), ("group", ctypes.c_int32), ("clip_alpha", ctypes.c_float),
         ("outlier_frac", ctypes.c_float), ("rank", ctypes.c_int32), ("adapter_bits", ctypes.c_int32),
-        ("adapter_group", ctypes.c_int32), ("flags", ctypes.c_uint32), ("reserved", ctypes.c_int32 * 5),
+        ("adapter_group", ctypes.c_int32), ("flags", ctypes.c_uint32), ("salient_channels", ctypes.c_int32),
+        ("salient_log2", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3),
     ]
 
 
@@ -78,7 +79,8 @@ def lib():
         L.cql_version.restype = I32
         L.cql_packed_layout.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(cql_layout)]
         L.cql_pack_workspace_size.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(U64)]
-        L.pack_compressed_weight.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, U64, P, U64, P]
+        L.pack_compressed_weight.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, U64, P, U64,
+                                             P]
         L.cql_workspace_size.argtypes = [ctypes.POINTER(cql_desc), I32, ctypes.POINTER(U64)]
         L.cql_workspace_init.argtypes = [P, U64, P]
         L.compressed_linear_forward.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P, ctypes.c_int,
@@ -115,11 +117,13 @@ def _check(st: int, where: str):
 
 
 def make_desc(n_out: int, k_in: int, mask: int = CQL_MASK_2_4, codec: int = CQL_CODEC_INT4_SYM,
-              clip_alpha: float = 0.9, outlier_frac: float = 0.0, rank: int = 0, flags: int = 0) -> cql_desc:
+              clip_alpha: float = 0.9, outlier_frac: float = 0.0, rank: int = 0, flags: int = 0,
+              salient_channels: int = 0, salient_log2: int = 0) -> cql_desc:
     d = cql_desc()
     d.n_out, d.k_in, d.mask, d.codec, d.group = n_out, k_in, mask, codec, 128
     d.clip_alpha, d.outlier_frac, d.rank = clip_alpha, outlier_frac, rank
     d.adapter_bits, d.adapter_group, d.flags = 4, 128, flags
+    d.salient_channels, d.salient_log2 = salient_channels, salient_log2
     return d
 
 
@@ -147,9 +151,11 @@ def cql_pack_workspace_size(desc: cql_desc) -> int:
     return int(v.value)
 
 
-def pack_compressed_weight(desc, W, w_dt, L, R, packed, packed_bytes, workspace, ws_bytes, stream=None):
-    _check(lib().pack_compressed_weight(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(L), _ptr(R), _ptr(packed),
-                                        int(packed_bytes), _ptr(workspace), int(ws_bytes), _stream(stream)),
+def pack_compressed_weight(desc, W, w_dt, L, R, act_absmean, packed, packed_bytes, workspace, ws_bytes,
+                           stream=None):
+    _check(lib().pack_compressed_weight(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(L), _ptr(R), _ptr(act_absmean),
+                                        _ptr(packed), int(packed_bytes), _ptr(workspace), int(ws_bytes),
+                                        _stream(stream)),
            "pack_compressed_weight")
 
 
@@ -198,11 +204,12 @@ class CompressedLinear:
     """Packs one layer on the GPU and runs its forward pass.
 
     ``W`` is a CUDA tensor [N][K] (fp32 or bf16), ``L`` [N][r] and ``R`` [r][K]
-    fp32 CUDA tensors (or None when rank is 0).  Buffers are torch tensors
-    allocated once; forward calls allocate only the output tensor (or write
-    into ``out``)."""
+    fp32 CUDA tensors (or None when rank is 0), ``act_absmean`` a fp32 CUDA
+    tensor [K] of per-channel mean |x| (SLiM^O layers only).  Buffers are
+    torch tensors allocated once; forward calls allocate only the output
+    tensor (or write into ``out``)."""
 
-    def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None):
+    def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None, act_absmean=None):
         import torch
         self.desc = desc
         self.layout = cql_packed_layout(desc)
@@ -211,8 +218,9 @@ class CompressedLinear:
         pw = cql_pack_workspace_size(desc)
         pws = torch.empty(max(pw, 256), dtype=torch.uint8, device=dev)
         pack_compressed_weight(desc, W.contiguous(), _dt_of(W), None if L is None else L.contiguous(),
-                               None if R is None else R.contiguous(), self.packed, self.layout.total_bytes,
-                               pws, pw, stream)
+                               None if R is None else R.contiguous(),
+                               None if act_absmean is None else act_absmean.contiguous(), self.packed,
+                               self.layout.total_bytes, pws, pw, stream)
         self._pack_ws = pws            # kept alive until the pack kernels ran
         self._ws = {}
 

@@ -22,6 +22,9 @@ cql_status validate_desc(const cql_desc* d) {
   if (!(d->clip_alpha > 0.0f && d->clip_alpha <= 1.0f)) return CQL_ERR_ARG;
   if (!(d->outlier_frac >= 0.0f && d->outlier_frac <= 0.0625f)) return CQL_ERR_ARG;
   if (d->rank < 0 || d->rank > 256 || d->rank % 16 != 0) return CQL_ERR_ARG;
+  if (d->salient_channels < 0 || d->salient_channels > d->k_in / 8) return CQL_ERR_ARG;
+  if (d->salient_channels > 0 ? (d->salient_log2 < 1 || d->salient_log2 > 8) : d->salient_log2 != 0)
+    return CQL_ERR_ARG;
   if (codec_is_lut(d->codec)) {
     if (d->mask != CQL_MASK_NONE) return CQL_ERR_UNSUPPORTED;
     if (d->k_in > 16384) return CQL_ERR_UNSUPPORTED;          // per-row sort lives in shared memory
@@ -56,6 +59,7 @@ void compute_layout(const cql_desc& d, cql_layout* L) {
     len[CQL_PLANE_L_VALUES] = n * rb.l_values;
     len[CQL_PLANE_L_SCALES] = 2 * (n / 128) * r;
   }
+  len[CQL_PLANE_SALIENT] = 2 * (uint64_t)d.salient_channels;
   uint64_t pos = 0;
   for (int i = 0; i < CQL_NPLANES; ++i) {
     pos = align256(pos);
@@ -78,7 +82,8 @@ HeaderBytes make_header(const cql_desc& d, const cql_layout& L) {
   memcpy(b + 72, &L.total_bytes, 8);
   memcpy(b + 80, &L.nnz, 8);
   memcpy(b + 88, L.off, 8 * CQL_NPLANES);
-  memcpy(b + 184, L.len, 8 * CQL_NPLANES);
+  memcpy(b + 88 + 8 * CQL_NPLANES, L.len, 8 * CQL_NPLANES);
+  static_assert(88 + 16 * CQL_NPLANES <= CQL_HEADER_BYTES, "header size");
   return h;
 }
 
@@ -105,6 +110,11 @@ PackWorkspace pack_workspace_layout(const cql_desc& d) {
   w.tiecnt = pos;    pos = align256(pos + nblk * 4);
   w.tieoff = pos;    pos = align256(pos + (nblk + 1) * 4);
   w.row_counts = pos; pos = align256(pos + (uint64_t)d.n_out * 4);
+  const bool sal = d.salient_channels > 0;
+  w.w_scaled = pos;  pos = align256(pos + (sal ? total * 4 : 0));
+  w.sal_partial = pos; pos = align256(pos + (sal ? (uint64_t)(d.n_out / 64) * d.k_in * 8 : 0));
+  w.sal = pos;       pos = align256(pos + (sal ? (uint64_t)d.k_in * 8 : 0));
+  w.sal_flag = pos;  pos = align256(pos + (sal ? (uint64_t)d.k_in : 0));
   w.total = pos;
   return w;
 }
@@ -122,6 +132,7 @@ ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch) {
   w.y_acc = pos;     pos = align256(pos + (batch <= CQL_MAX_DECODE_BATCH ? (uint64_t)batch * n * 4 : 0));
   w.t_part = pos;    pos = align256(pos + upr * bp * rpad * 4);
   w.t_final = pos;   pos = align256(pos + 2 * bp * rpad * 4);   // two t buffers, alternating by call
+  w.xs = pos;        pos = align256(pos + (d.salient_channels > 0 ? (uint64_t)batch * d.k_in * 2 : 0));
   w.prefill = pos;
   if (batch > CQL_MAX_DECODE_BATCH) pos = align256(pos + prefill_layout(d, batch).total);
   w.total = pos;
@@ -165,7 +176,7 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes) {
 }
 
 cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt, const float* L,
-                                  const float* R, void* packed, uint64_t packed_bytes, void* workspace,
+                                  const float* R, const float* act_absmean, void* packed, uint64_t packed_bytes, void* workspace,
                                   uint64_t ws_bytes, cql_stream_t stream) {
   cql_status s = validate_desc(desc);
   if (s != CQL_OK) return s;
@@ -175,6 +186,8 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
   if (d.rank > 0 && (L == nullptr || R == nullptr)) return CQL_ERR_ARG;
   if (!aligned(W, 16) || !aligned(packed, 256) || !aligned(workspace, 256)) return CQL_ERR_ALIGN;
   if (d.rank > 0 && (!aligned(L, 16) || !aligned(R, 16))) return CQL_ERR_ALIGN;
+  if (d.salient_channels > 0 && act_absmean == nullptr) return CQL_ERR_ARG;
+  if (d.salient_channels > 0 && !aligned(act_absmean, 4)) return CQL_ERR_ALIGN;
   cql_layout lay;
   compute_layout(d, &lay);
   if (packed_bytes < lay.total_bytes) return CQL_ERR_SIZE;
@@ -211,6 +224,12 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
   p.topk_tiecnt = reinterpret_cast<uint32_t*>(ws + pw.tiecnt);
   p.topk_tieoff = reinterpret_cast<uint32_t*>(ws + pw.tieoff);
   p.row_counts = reinterpret_cast<uint32_t*>(ws + pw.row_counts);
+  p.act_absmean = act_absmean;
+  p.salient = reinterpret_cast<uint16_t*>(base + lay.off[CQL_PLANE_SALIENT]);
+  p.w_scaled = reinterpret_cast<float*>(ws + pw.w_scaled);
+  p.sal_partial = reinterpret_cast<double*>(ws + pw.sal_partial);
+  p.sal = reinterpret_cast<double*>(ws + pw.sal);
+  p.sal_flag = ws + pw.sal_flag;
   if (d.outlier_frac <= 0.0f) p.csr_rowptr = nullptr;
   const HeaderBytes h = make_header(d, lay);
   const cudaError_t e = launch_pack(p, h, lay.total_bytes, reinterpret_cast<cudaStream_t>(stream));
@@ -285,6 +304,13 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   p.counters = reinterpret_cast<uint32_t*>(ws + fw.counters);
   p.t_part = reinterpret_cast<float*>(ws + fw.t_part);
   p.t_final = reinterpret_cast<float*>(ws + fw.t_final);
+  if (d.salient_channels > 0) {
+    // SLiM^O: every later step reads x' from the workspace
+    const cudaError_t e0 = launch_salient_x(p, reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_SALIENT]),
+                                            ws + fw.xs, reinterpret_cast<cudaStream_t>(stream));
+    if (e0 != cudaSuccess) return CQL_ERR_CUDA;
+    p.x = ws + fw.xs;
+  }
   const cudaError_t e = batch > CQL_MAX_DECODE_BATCH
                             ? launch_prefill(p, ws + fw.prefill, reinterpret_cast<cudaStream_t>(stream))
                             : launch_decode(p, reinterpret_cast<cudaStream_t>(stream));

@@ -47,12 +47,23 @@ struct PackParams {
   uint32_t* topk_tiecnt;             // [nblk]
   uint32_t* topk_tieoff;             // [nblk+1]
   uint32_t* row_counts;              // [N]
+  // SLiM^O (salient_channels > 0): input statistic, output plane, scratch
+  const float* act_absmean;          // [K] mean |x_c|
+  uint16_t* salient;                 // SALIENT plane [m]
+  float* w_scaled;                   // [N*K] W' (fp32)
+  double* sal_partial;               // [N/64][K]
+  double* sal;                       // [K]
+  uint8_t* sal_flag;                 // [K]
 };
 
 struct PackWorkspace {
-  uint64_t out_bits, state, hist, tiecnt, tieoff, row_counts, total;
+  uint64_t out_bits, state, hist, tiecnt, tieoff, row_counts, w_scaled, sal_partial, sal, sal_flag, total;
 };
 PackWorkspace pack_workspace_layout(const cql_desc& d);
+
+// SLiM^O packer step: selects the salient channels (SALIENT plane) and
+// writes W' into the workspace; on return p.W / p.wdt name W' (fp32).
+cudaError_t launch_salient_pack(PackParams& p, cudaStream_t st);
 
 cudaError_t launch_pack(const PackParams& p, const HeaderBytes& hdr, uint64_t total_bytes,
                         cudaStream_t st);
@@ -98,7 +109,7 @@ struct DecodeParams {
 };
 
 struct ForwardWorkspace {
-  uint64_t err, t_counter, y_acc, counters, t_part, t_final, prefill, total;
+  uint64_t err, t_counter, y_acc, counters, t_part, t_final, xs, prefill, total;
 };
 ForwardWorkspace forward_workspace_layout(const cql_desc& d, int batch);
 
@@ -107,10 +118,15 @@ CQL_DEV bool header_ok(const DecodeParams& p) {
   const uint32_t* h = reinterpret_cast<const uint32_t*>(p.header);
   const int32_t* d = reinterpret_cast<const int32_t*>(p.header + 8);
   return h[0] == 0x314C5143u /* "CQL1" */ && h[1] == CQL_VERSION && d[0] == p.d.n_out && d[1] == p.d.k_in &&
-         d[2] == p.d.mask && d[3] == p.d.codec && d[7] == p.d.rank;
+         d[2] == p.d.mask && d[3] == p.d.codec && d[7] == p.d.rank && d[11] == p.d.salient_channels &&
+         d[12] == p.d.salient_log2;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+// SLiM^O forward prologue: xs = x with the listed channels divided by
+// 2^salient_log2 (same dtype, [batch][K]); PDL-chained to the kernel before.
+cudaError_t launch_salient_x(const DecodeParams& p, const uint16_t* list, void* xs, cudaStream_t st);
 
 // Device address of compressed_linear_forward_noalloc's scratch array on the
 // current device (nullptr before its first call there).

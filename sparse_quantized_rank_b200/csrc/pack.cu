@@ -502,6 +502,7 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
   cudaError_t e = cudaMemsetAsync(p.packed, 0, total_bytes, st);
   if (e != cudaSuccess) return e;
   k_write_header<<<1, 64, 0, st>>>(hdr, p.packed);
+  if (p.d.salient_channels > 0 && (e = launch_salient_pack(p, st)) != cudaSuccess) return e;
 
   const uint64_t total = (uint64_t)N * K;
   if (p.nnz_target > 0) {

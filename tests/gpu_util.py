@@ -12,7 +12,8 @@ DT_NAME = {C.CQL_DT_F32: "f32", C.CQL_DT_F16: "f16", C.CQL_DT_BF16: "bf16"}
 
 
 def c_desc(od: O.OracleDesc, flags: int = 0):
-    return C.make_desc(od.n_out, od.k_in, od.mask, od.codec, od.clip_alpha, od.outlier_frac, od.rank, flags)
+    return C.make_desc(od.n_out, od.k_in, od.mask, od.codec, od.clip_alpha, od.outlier_frac, od.rank, flags,
+                       od.salient_channels, od.salient_log2)
 
 
 def device_inputs(inp, wl, dev):
@@ -36,10 +37,12 @@ class Case:
         self.wl = wl
         self.inp = make_layer_inputs(wl, max_batch=max_batch)
         self.od = O.desc_for(wl)
-        self.parts = O.compress(self.od, self.inp["w"], self.inp["L"], self.inp["R"])
+        self.parts = O.compress(self.od, self.inp["w"], self.inp["L"], self.inp["R"], self.inp["act_absmean"])
         self.ref_bytes = O.pack_bytes(self.od, self.parts)
         self.W, self.L, self.R, self.x = device_inputs(self.inp, wl, dev)
-        self.layer = C.CompressedLinear(c_desc(self.od), self.W, self.L, self.R)
+        act = self.inp["act_absmean"]
+        self.act = None if act is None else torch.from_numpy(act).to(dev)
+        self.layer = C.CompressedLinear(c_desc(self.od), self.W, self.L, self.R, act_absmean=self.act)
         torch.cuda.synchronize()
 
     def packed_bytes(self):

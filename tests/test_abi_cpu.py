@@ -34,13 +34,13 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) == set(C.EXPORTED), names
     for n in names:
         assert hasattr(lib, n), n
-    assert C.cql_version() == 1
+    assert C.cql_version() == O.FORMAT_VERSION == 2
     assert C.cql_status_string(C.CQL_ERR_SIZE).startswith("CQL_ERR_SIZE")
 
 
 def test_desc_struct_size():
     assert ctypes.sizeof(C.cql_desc) == 64
-    assert ctypes.sizeof(C.cql_layout) == 16 + 2 * 8 * 12
+    assert ctypes.sizeof(C.cql_layout) == 16 + 2 * 8 * 13
 
 
 DESCS = [
@@ -51,6 +51,8 @@ DESCS = [
     dict(n_out=128, k_in=384, mask=1, codec=1, rank=48),
     dict(n_out=384, k_in=256, mask=0, codec=3, outlier_frac=0.01, rank=32),
     dict(n_out=128, k_in=128, mask=2, codec=0, outlier_frac=0.001),
+    dict(n_out=11008, k_in=4096, mask=1, codec=0, rank=128, salient_channels=41, salient_log2=1),
+    dict(n_out=256, k_in=1024, mask=0, codec=2, outlier_frac=0.01, salient_channels=128, salient_log2=8),
 ]
 
 
@@ -59,7 +61,8 @@ def test_layout_matches_oracle(lib, kw):
     d = C.make_desc(**kw)
     lay = C.cql_packed_layout(d)
     od = O.OracleDesc(kw["n_out"], kw["k_in"], kw["mask"], kw["codec"], 0.9, kw.get("outlier_frac", 0.0),
-                      kw.get("rank", 0))
+                      kw.get("rank", 0), salient_channels=kw.get("salient_channels", 0),
+                      salient_log2=kw.get("salient_log2", 0))
     ol = O.packed_layout(od)
     assert list(lay.off) == ol["off"]
     assert list(lay.len) == ol["len"]
@@ -81,6 +84,11 @@ def test_descriptor_validation(lib):
         (dict(ok, outlier_frac=-0.1), C.CQL_ERR_ARG),
         (dict(ok, codec=2), C.CQL_ERR_UNSUPPORTED),          # LUT needs no mask
         (dict(ok, mask=0, codec=2, k_in=32768), C.CQL_ERR_UNSUPPORTED),
+        (dict(ok, salient_channels=-1, salient_log2=1), C.CQL_ERR_ARG),
+        (dict(ok, salient_channels=65, salient_log2=1), C.CQL_ERR_ARG),     # more than K/8
+        (dict(ok, salient_channels=5, salient_log2=0), C.CQL_ERR_ARG),      # factor 1 is no scaling
+        (dict(ok, salient_channels=5, salient_log2=9), C.CQL_ERR_ARG),
+        (dict(ok, salient_channels=0, salient_log2=1), C.CQL_ERR_ARG),      # factor without channels
     ]
     for kw, st in bad:
         with pytest.raises(C.CqlError) as ei:
@@ -113,15 +121,21 @@ def test_call_errors_return_before_launch(lib):
     st = L.compressed_linear_forward(ctypes.byref(d), fake, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 0, fake, ws, None)
     assert st == C.CQL_ERR_ARG
     pw = C.cql_pack_workspace_size(d)
-    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, None, None, fake, lay.total_bytes, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, None, None, None, fake, lay.total_bytes, fake, pw,
                                   None)
     assert st == C.CQL_ERR_ARG                       # rank 16 needs L and R
-    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, fake, fake, fake, lay.total_bytes - 1, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, fake, fake, None, fake, lay.total_bytes - 1, fake, pw,
                                   None)
     assert st == C.CQL_ERR_SIZE
-    st = L.pack_compressed_weight(ctypes.byref(d), fake + 8, C.CQL_DT_F32, fake, fake, fake, lay.total_bytes, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake + 8, C.CQL_DT_F32, fake, fake, None, fake, lay.total_bytes, fake, pw,
                                   None)
     assert st == C.CQL_ERR_ALIGN
+    ds = C.make_desc(256, 512, rank=16, salient_channels=5, salient_log2=1)
+    lay_s = C.cql_packed_layout(ds)
+    pws = C.cql_pack_workspace_size(ds)
+    st = L.pack_compressed_weight(ctypes.byref(ds), fake, C.CQL_DT_F32, fake, fake, None, fake, lay_s.total_bytes,
+                                  fake, pws, None)
+    assert st == C.CQL_ERR_ARG                       # SLiM^O needs the activation statistic
     assert L.cql_get_device_status(None, None, None) == C.CQL_ERR_ARG
 
 

@@ -414,10 +414,16 @@ def _brute_forward(parts, desc, x):
                     rv = float(parts["R_q"][t, j]) * float(parts["R_s"][t, j // 128])
                     acc += lv * rv
                 W[i][j] += acc
+    # SLiM^O: the matrix above acts on x with the salient channels divided
+    # by the factor; equivalently its salient columns are divided by it
+    div = [1.0] * k
+    for c in parts.get("salient", []):
+        div[int(c)] = float(2 ** int(desc.salient_log2))
     y = np.zeros((x.shape[0], n))
     for b in range(x.shape[0]):
         for i in range(n):
-            y[b, i] = math.fsum(W[i][j] * float(x[b, j]) for j in range(k))
+            y[b, i] = math.fsum(W[i][j] * (float(x[b, j]) / div[j]) for j in range(k))
+    W = [[W[i][j] / div[j] for j in range(k)] for i in range(n)]
     return y, np.array(W)
 
 
@@ -425,12 +431,13 @@ def _brute_forward(parts, desc, x):
     ("tiny", dict(n=128, k=256, rank=16)),
     ("down_unstructured", dict(n=128, k=256, rank=32, codec="int3")),
     ("lut_dense_sparse", dict(n=128, k=256)),
+    ("mlp_up_slimo", dict(n=128, k=256, rank=16, salient_channels=4, salient_log2=2)),
 ])
 def test_forward_matches_brute_force(name, over):
     wl = workload(name, **over)
     inp = make_layer_inputs(wl, max_batch=2)
     d = O.desc_for(wl)
-    parts = O.compress(d, inp["w"], inp["L"], inp["R"])
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
     y = O.forward(parts, inp["x"])
     yb, Wb = _brute_forward(parts, d, inp["x"])
     assert O.rel_err(y, yb) < 1e-12
