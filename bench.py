@@ -121,24 +121,30 @@ def kernels_per_step(wl, batch):
     the CUDA-core paths add a pre-kernel when there are adapters or outliers;
     a SLiM^O layer adds the activation-scaling prologue."""
     pro = 1 if wl.salient_channels else 0
+    if batch > 16:                       # prefill: adapter passes (4 kernels) and the main GEMM
+        return pro + 1 + (4 if wl.rank else 0) + (0 if (wl.mask == "2:4" and wl.codec == "int4") else 1)
     if wl.mask == "2:4" and wl.codec == "int4":
         return 2 + pro
     return 2 + pro + (1 if (wl.rank or wl.outlier_frac) else 0)
 
 
-def source_hash():
-    """Hash of the sources k_decode_tc is compiled from (the kernel and its
-    launch, and the device helpers it includes)."""
+DECODE_SOURCES = ("decode_tc.cu", "tc.cuh", "common.cuh")
+PREFILL_SOURCES = ("prefill_sp.cu", "tc.cuh", "common.cuh")
+
+
+def source_hash(files=DECODE_SOURCES):
+    """Hash of the sources a profiled kernel is compiled from (the kernel and
+    its launch, and the device helpers it includes)."""
     h = hashlib.sha256()
-    for f in ("decode_tc.cu", "tc.cuh", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "sparse_quantized_rank_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(name):
+def profiled_traffic(name, files=DECODE_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, or None when the
-    decode sources changed since the counters were taken."""
+    kernel's sources changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", f"{name}.md")
     if not os.path.exists(p):
         return None
@@ -146,9 +152,11 @@ def profiled_traffic(name):
     if not m:
         return None
     d = json.loads(m.group(1))
-    if d.get("source_hash") != source_hash():
+    if d.get("source_hash") != source_hash(files):
         return None
-    return d.get("dram_bytes_per_launch")
+    if "dram_bytes_per_launch" in d:
+        return d["dram_bytes_per_launch"]
+    return d.get("dram_bytes_read_per_launch", 0) + d.get("dram_bytes_write_per_launch", 0)
 
 
 class ClockSampler:
@@ -454,6 +462,22 @@ def run_cql(args):
         "gpu_launches": args.steps * b.kernels_per_step,
         "clocks": clocks,
     }
+    if args.batch > C.CQL_MAX_DECODE_BATCH:
+        # prefill: a contraction on the sparse tensor cores
+        tf_peak, tf_src = measured_tflops()
+        dense = 2.0 * args.batch * wl.n * wl.k
+        algo = dense / 2 + 2.0 * args.batch * wl.rank * (wl.n + wl.k)
+        line["roofline"] = {
+            "bound": "tensor", "achieved": dense / per_step / 1e12, "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": dense / per_step / 1e12 / tf_peak,
+            "traffic": profiled_traffic(f"{wl.name}_b{args.batch}", PREFILL_SOURCES),
+            "peak_source": f"{tf_src} dense bf16 (MEASURED_PEAKS.json bf16_tflops)",
+            "kernel": "k_pf_sgemm (tcgen05.mma.sp, codes converted on chip) after the adapter passes; achieved = "
+                      "dense-equivalent 2MNK per call / whole-call time",
+            "sparse_frac": algo / per_step / 1e12 / (2 * tf_peak),
+            "sparse_note": "algorithmic flops (MNK on the kept half plus the adapter product) against twice the "
+                           "dense peak (the sparse tensor-core rate)"}
+        line["kernels_per_step"] = "k_pf_dequant_l, k_pf_dequant_r, k_pf_gemm (T), k_pf_tsplit, k_pf_sgemm"
     del b
     torch.cuda.empty_cache()
     if rank == 0 and world == 1:
