@@ -17,6 +17,11 @@ Sources (web pages summarising the methods):
 * SqueezeLLM: Dense-and-Sparse Quantization -- "Approach" (non-uniform LUT
   quantisation; the top 0.45% outliers go to a full-precision CSR matrix so
   the dense part has a narrower range).
+* SLiM (same page), review summary "SLIM-LoRA" and rebuttal "Assumptions in
+  Theoretical Derivations": the adapters minimise the saliency-weighted
+  error norm ||F(W - W_C - L R)|| for an additive, invertible saliency F
+  built from the layer's (positive) average input; the solution is the SVD
+  of F(W - W_C), mapped back through F^-1.  Naive-LoRA is the plain SVD.
 * SLiM (same page), rebuttal "Output Error Minimization in SLiM-Quant": the
   output-error variant scales the weights of the ~1% most salient input
   channels up by a factor and the matching activations down by it; a
@@ -55,6 +60,7 @@ __all__ = [
     "quantize_adapter_rows", "quantize_adapter_cols",
     "build_csr", "compress", "packed_layout", "pack_bytes",
     "channel_saliency", "select_salient_channels", "scale_activations",
+    "compressed_matrix", "slim_lora", "lowrank_objective", "build_adapters",
     "forward", "forward_terms", "dense_reconstruction",
     "rel_err", "pack_and_forward", "HEADER_BYTES", "NPLANES",
     "P_HEADER", "P_VALUES", "P_META", "P_SCALES", "P_VOFF", "P_CSR_ROWPTR",
@@ -528,6 +534,75 @@ def dense_reconstruction(parts: Dict[str, np.ndarray]) -> np.ndarray:
         sal = parts["salient"]
         wd[:, sal] = wd[:, sal] / float(2 ** int(parts["salient_log2"]))
     return wd
+
+
+# ---------------------------------------------------------------------------
+# adapter construction (SLiM review summary, "SLIM-LoRA"; rebuttal,
+# "Assumptions in Theoretical Derivations")
+# ---------------------------------------------------------------------------
+
+def compressed_matrix(parts: Dict[str, np.ndarray]) -> np.ndarray:
+    """W_C: what the sparse quantised part and the CSR outliers represent,
+    in the space the codec encoded (W' for a SLiM^O layer), fp64.  The
+    adapters are built to compensate W(') - W_C."""
+    wd = parts["w_dense"].copy()
+    if "csr_row_ptr" in parts:
+        rp, col, val = parts["csr_row_ptr"], parts["csr_col"], parts["csr_val"]
+        rows = np.repeat(np.arange(len(rp) - 1), np.diff(rp))
+        np.add.at(wd, (rows, col), val)
+    return wd
+
+
+def slim_lora(err: np.ndarray, rank: int, act_absmean: Optional[np.ndarray] = None):
+    """Rank-r adapters (L [N][r], R [r][K]) of the compression error
+    E = W - W_C.
+
+    SLiM-LoRA: with F(M) = M diag(xbar) (xbar the layer's average input
+    magnitude, positive, so F is additive and invertible), minimise
+    ||F(E - L R)||_F; by Eckart-Young the optimum is L R = F^-1((F(E))_r),
+    (.)_r the rank-r truncated SVD.  Reading of the garbled formulas: F
+    scales the input columns by xbar, and the singular values are split as
+    L = U_r Sigma_r^(1/2), R = Sigma_r^(1/2) V_r^T diag(xbar)^-1 (the page
+    fixes only the product).  Naive-LoRA (act_absmean None): xbar = 1."""
+    e = np.asarray(err, dtype=np.float64)
+    k = e.shape[1]
+    xbar = np.ones(k) if act_absmean is None else np.asarray(act_absmean, dtype=np.float32).astype(np.float64)
+    assert (xbar > 0).all()
+    u, sv, vt = np.linalg.svd(e * xbar[None, :], full_matrices=False)
+    root = np.sqrt(sv[:rank])
+    L = u[:, :rank] * root[None, :]
+    R = (root[:, None] * vt[:rank]) / xbar[None, :]
+    return L, R
+
+
+def build_adapters(desc: OracleDesc, w: np.ndarray, act_absmean: Optional[np.ndarray] = None,
+                   naive: bool = False):
+    """SLiM-LoRA (or Naive-LoRA) adapters of rank desc.rank for W.
+
+    Compresses W without adapters (every encoding step but the last), forms
+    E = W(') - W_C in the space the codec encoded, and returns slim_lora(E).
+    The saliency weight is the average input the adapters see: act_absmean,
+    divided by the factor on a SLiM^O layer's salient channels (reading)."""
+    d0 = OracleDesc(desc.n_out, desc.k_in, desc.mask, desc.codec, desc.clip_alpha, desc.outlier_frac, 0,
+                    salient_channels=desc.salient_channels, salient_log2=desc.salient_log2)
+    parts = compress(d0, w, act_absmean=act_absmean)
+    wp = np.array(w, dtype=np.float64, copy=True)
+    xbar = None if act_absmean is None else np.asarray(act_absmean, dtype=np.float32).astype(np.float64)
+    if "salient" in parts:
+        f = float(2 ** desc.salient_log2)
+        wp[:, parts["salient"]] *= f
+        if xbar is not None:
+            xbar[parts["salient"]] /= f
+    err = wp - compressed_matrix(parts)
+    return slim_lora(err, desc.rank, None if naive else xbar)
+
+
+def lowrank_objective(err: np.ndarray, L: np.ndarray, R: np.ndarray, act_absmean=None) -> float:
+    """||F(E - L R)||_F^2 with F as in slim_lora."""
+    e = np.asarray(err, dtype=np.float64)
+    xbar = np.ones(e.shape[1]) if act_absmean is None else np.asarray(act_absmean, dtype=np.float32).astype(np.float64)
+    d = (e - np.asarray(L, dtype=np.float64) @ np.asarray(R, dtype=np.float64)) * xbar[None, :]
+    return float(np.sum(d * d))
 
 
 def rel_err(y: np.ndarray, ref: np.ndarray) -> float:

@@ -609,3 +609,109 @@ def test_slimo_reduces_the_error_of_the_salient_channels():
     err_s = np.abs(O.dense_reconstruction(ps)[:, sal] - w[:, sal]).mean()
     err_p = np.abs(O.dense_reconstruction(pp)[:, sal] - w[:, sal]).mean()
     assert err_s < 0.85 * err_p, (err_s, err_p)
+
+
+# ---------------------------------------------------------------------------
+# SLiM-LoRA / Naive-LoRA adapter construction (SLiM review summary,
+# "SLIM-LoRA"; rebuttal, "Assumptions in Theoretical Derivations")
+# ---------------------------------------------------------------------------
+
+def test_naive_lora_is_the_truncated_svd_by_eigh():
+    """Naive-LoRA's L R is the best rank-r approximation of E; rebuilt here
+    from the top-r eigenvectors of E^T E (numpy.linalg.eigh, not svd)."""
+    rng = np.random.default_rng(21)
+    e = rng.standard_normal((96, 64)) * np.linspace(2.0, 0.1, 64)[None, :]
+    L, R = O.slim_lora(e, 8)
+    lam, v = np.linalg.eigh(e.T @ e)
+    vr = v[:, np.argsort(lam)[::-1][:8]]
+    assert np.abs(L @ R - e @ vr @ vr.T).max() < 1e-10
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_lora_projection_identity(weighted):
+    """F(L R) is the orthogonal projection of F(E) onto a rank-r subspace, so
+    ||F(E - L R)||^2 = ||F(E)||^2 - ||F(L R)||^2 (Pythagoras)."""
+    rng = np.random.default_rng(22)
+    e = rng.standard_normal((80, 48))
+    a = np.exp(rng.standard_normal(48)).astype(np.float32) if weighted else None
+    L, R = O.slim_lora(e, 6, a)
+    xb = np.ones(48) if a is None else a.astype(np.float64)
+    fe, flr = e * xb, (L @ R) * xb
+    obj = O.lowrank_objective(e, L, R, a)
+    assert abs(obj - (np.sum(fe * fe) - np.sum(flr * flr))) <= 1e-9 * np.sum(fe * fe)
+
+
+def test_lora_recovers_an_exact_low_rank_error():
+    rng = np.random.default_rng(23)
+    e = rng.standard_normal((64, 5)) @ rng.standard_normal((5, 96))
+    a = np.exp(rng.standard_normal(96)).astype(np.float32)
+    for act in (None, a):
+        L, R = O.slim_lora(e, 5, act)
+        assert L.shape == (64, 5) and R.shape == (5, 96)
+        assert np.abs(L @ R - e).max() < 1e-10 * np.abs(e).max()
+
+
+def test_saliency_changes_which_error_is_kept():
+    """Closed form: E diagonal, rank 1.  Naive-LoRA keeps the largest |d_i|;
+    SLiM-LoRA keeps the largest |d_i xbar_i|, and maps it back exactly."""
+    d = np.array([3.0, -1.0, 2.0, 0.5])
+    e = np.diag(d)
+    xbar = np.array([1.0, 8.0, 1.0, 1.0], dtype=np.float32)
+    L, R = O.slim_lora(e, 1)
+    exp = np.zeros((4, 4))
+    exp[0, 0] = 3.0
+    assert np.abs(L @ R - exp).max() < 1e-12
+    L, R = O.slim_lora(e, 1, xbar)
+    exp = np.zeros((4, 4))
+    exp[1, 1] = -1.0
+    assert np.abs(L @ R - exp).max() < 1e-12
+
+
+def test_slim_lora_beats_naive_on_its_own_objective():
+    rng = np.random.default_rng(24)
+    e = rng.standard_normal((128, 96))
+    a = np.exp(rng.standard_normal(96)).astype(np.float32)
+    Ls, Rs = O.slim_lora(e, 10, a)
+    Ln, Rn = O.slim_lora(e, 10)
+    assert O.lowrank_objective(e, Ls, Rs, a) < O.lowrank_objective(e, Ln, Rn, a)
+    assert O.lowrank_objective(e, Ln, Rn) < O.lowrank_objective(e, Ls, Rs)
+    # a constant factor on xbar leaves the adapters' product unchanged
+    L2, R2 = O.slim_lora(e, 10, (a * 4).astype(np.float32))
+    assert np.abs(L2 @ R2 - Ls @ Rs).max() < 1e-10
+
+
+def test_build_adapters_compensates_the_compression_error():
+    """Wiring: E is W minus what the codes and the CSR represent; adding the
+    adapters' product shrinks the weighted error by exactly their share, and
+    the adapters built by build_adapters are the ones slim_lora gives for an
+    independently formed E (dense reconstruction of a rank-0 layer)."""
+    wl = workload("tiny", n=128, k=256, rank=0, outlier_frac=0.01)
+    inp = make_layer_inputs(wl, max_batch=1)
+    d = O.desc_for(wl)
+    d.rank = 16
+    act = np.exp(0.5 * np.random.default_rng(3).standard_normal(256)).astype(np.float32)
+    L, R = O.build_adapters(d, inp["w"], act)
+    d0 = O.desc_for(wl)
+    p0 = O.compress(d0, inp["w"])
+    e = inp["w"].astype(np.float64) - O.dense_reconstruction(p0)
+    L2, R2 = O.slim_lora(e, 16, act)
+    assert np.abs(L @ R - L2 @ R2).max() < 1e-12
+    assert O.lowrank_objective(e, L, R, act) < O.lowrank_objective(e, np.zeros((128, 1)), np.zeros((1, 256)), act)
+
+
+def test_build_adapters_on_a_slimo_layer_match_the_original_space():
+    """On a SLiM^O layer the adapters act on x' = x / sigma, so L R diag(1/sigma)
+    must be the SLiM-LoRA solution for the original-space error W - W_hat with
+    the original statistic (the weighted norms coincide)."""
+    wl = workload("mlp_up_slimo", n=128, k=512, rank=0, salient_channels=8, salient_log2=2)
+    inp = make_layer_inputs(wl, max_batch=1)
+    d = O.desc_for(wl)
+    d.rank = 16
+    L, R = O.build_adapters(d, inp["w"], inp["act_absmean"])
+    d0 = O.desc_for(wl)
+    p0 = O.compress(d0, inp["w"], act_absmean=inp["act_absmean"])
+    e = inp["w"].astype(np.float64) - O.dense_reconstruction(p0)
+    L2, R2 = O.slim_lora(e, 16, inp["act_absmean"])
+    div = np.ones(512)
+    div[p0["salient"]] = 4.0
+    assert np.abs((L @ R) / div[None, :] - L2 @ R2).max() < 1e-12
