@@ -533,6 +533,7 @@ def extra_lines(torch, C, dev, stream, barrier):
         del b
         torch.cuda.empty_cache()
     out.append(stack_line(torch, C, dev, stream))
+    out.append(adapter_build_line(torch, C, dev, stream))
     tf_peak, _ = measured_tflops()
     for name in ("prefill_up", "prefill_down"):
         wl = workload(name)
@@ -551,6 +552,39 @@ def extra_lines(torch, C, dev, stream, barrier):
         del b
         torch.cuda.empty_cache()
     return out
+
+
+def adapter_build_line(torch, C, dev, stream, reps=3):
+    """SLiM-LoRA adapter construction (cql_build_adapters) for the full-size
+    mlp_up layer (11008x4096, rank 128): one-time packer-side cost, timed
+    with CUDA events after one warm run."""
+    from workloads import make_layer_inputs, workload
+    wl = workload("mlp_up")
+    inp = make_layer_inputs(wl, max_batch=1)
+    W, _, _, _ = device_inputs(torch, inp, wl, dev)
+    d = desc_from_workload(C, wl)
+    act = torch.exp(0.5 * torch.randn(wl.k, generator=torch.Generator().manual_seed(9))).to(dev)
+    zL = torch.zeros(wl.n, wl.rank, device=dev)
+    zR = torch.zeros(wl.rank, wl.k, device=dev)
+    layer = C.CompressedLinear(d, W, zL, zR)
+    nb = C.cql_adapter_workspace_size(d)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    L = torch.empty(wl.n, wl.rank, device=dev)
+    R = torch.empty(wl.rank, wl.k, device=dev)
+    with torch.cuda.stream(stream):
+        C.cql_build_adapters(d, W, C._dt_of(W), layer.packed, act, L, R, ws, nb, stream)
+        stream.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            C.cql_build_adapters(d, W, C._dt_of(W), layer.packed, act, L, R, ws, nb, stream)
+        t1.record(stream)
+        stream.synchronize()
+    ms = t0.elapsed_time(t1) / reps
+    del layer, ws, W
+    torch.cuda.empty_cache()
+    return {"workload": "SLiM-LoRA adapter construction, mlp_up 11008x4096 rank 128 (subspace p=160, 6 iterations)",
+            "ms_per_layer": round(ms, 3), "note": "one-time, packer side; fp32 CUDA-core GEMMs over F(E)"}
 
 
 def stack_line(torch, C, dev, stream, passes=20):

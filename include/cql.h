@@ -233,6 +233,36 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
                                   uint64_t packed_bytes, void* workspace, uint64_t ws_bytes,
                                   cql_stream_t stream);
 
+/* Scratch bytes cql_build_adapters needs (about 4 N K bytes plus
+ * O((N + K) r) for the subspace).  Host only.  CQL_ERR_ARG unless
+ * 0 < rank <= min(N, K). */
+cql_status cql_adapter_workspace_size(const cql_desc* desc, uint64_t* bytes);
+
+/* SLiM-LoRA adapters of a packed layer (SLiM review summary, "SLIM-LoRA";
+ * rebuttal, "Assumptions in Theoretical Derivations"): L [N][r] and R [r][K]
+ * minimising ||(E - L R) diag(xbar)||_F, E = W' - W_C the compression error
+ * (W' the matrix the codec encoded, W_C what the codes and the CSR outliers
+ * represent), xbar the input the adapters see: act_absmean, divided by the
+ * SLiM^O factor on the salient channels.  act_absmean NULL: Naive-LoRA
+ * (xbar = 1, the plain truncated SVD of E).
+ *   desc      the layer's descriptor; rank r with 0 < r <= min(N, K).
+ *   W         device [N][K], w_dt CQL_DT_F32 or CQL_DT_BF16, 16-byte aligned:
+ *             the matrix packed into 'packed'.
+ *   packed    device, 256-byte aligned, a buffer pack_compressed_weight
+ *             wrote for W under desc (its adapter planes are not read: pack
+ *             with zero adapters, build, then pack again with L and R).
+ *   act_absmean  device fp32 [K], every entry > 0, or NULL.
+ *   L, R      device fp32 outputs, row-major [N][r] and [r][K].
+ *   workspace device, >= cql_adapter_workspace_size bytes, 256-byte aligned.
+ * Method: randomized subspace iteration on E diag(xbar) (p = r + 32 rounded
+ * up to 32 columns, 6 iterations, CholeskyQR2), then a Jacobi
+ * eigen-decomposition of the p x p Gram matrix.  The result approaches the
+ * exact truncated SVD as the singular-value gap at r grows; the split of
+ * the singular values is L = U Sigma^(1/2), R = Sigma^(1/2) V^T diag(xbar)^-1. */
+cql_status cql_build_adapters(const cql_desc* desc, const void* W, cql_dtype w_dt, const void* packed,
+                              const float* act_absmean, float* L, float* R, void* workspace, uint64_t ws_bytes,
+                              cql_stream_t stream);
+
 /* Workspace bytes compressed_linear_forward needs for this layer and batch.
  * Host only. */
 cql_status cql_workspace_size(const cql_desc* desc, int32_t batch, uint64_t* bytes);

@@ -36,6 +36,7 @@ EXPORTED = (
     "cql_status_string", "cql_version", "cql_packed_layout", "cql_pack_workspace_size",
     "pack_compressed_weight", "cql_workspace_size", "cql_workspace_init",
     "compressed_linear_forward", "cql_get_device_status", "compressed_linear_forward_noalloc",
+    "cql_adapter_workspace_size", "cql_build_adapters",
 )
 
 
@@ -88,6 +89,8 @@ def lib():
         L.cql_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.compressed_linear_forward_noalloc.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P,
                                                         ctypes.c_int, I32, P]
+        L.cql_adapter_workspace_size.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(U64)]
+        L.cql_build_adapters.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, P, U64, P]
         for fn in EXPORTED[2:]:
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -183,6 +186,18 @@ def compressed_linear_forward_noalloc(desc, packed, x, x_dt, y, y_dt, batch, str
            "compressed_linear_forward_noalloc")
 
 
+def cql_adapter_workspace_size(desc: cql_desc) -> int:
+    v = ctypes.c_uint64()
+    _check(lib().cql_adapter_workspace_size(ctypes.byref(desc), ctypes.byref(v)), "cql_adapter_workspace_size")
+    return int(v.value)
+
+
+def cql_build_adapters(desc, W, w_dt, packed, act_absmean, L, R, workspace, ws_bytes, stream=None):
+    _check(lib().cql_build_adapters(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(packed), _ptr(act_absmean), _ptr(L),
+                                    _ptr(R), _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "cql_build_adapters")
+
+
 def cql_get_device_status(workspace, stream=None) -> int:
     """Device error word of a workspace (None: the fixed scratch of the
     no-workspace entry point on the current device)."""
@@ -223,6 +238,28 @@ class CompressedLinear:
                                self.layout.total_bytes, pws, pw, stream)
         self._pack_ws = pws            # kept alive until the pack kernels ran
         self._ws = {}
+
+    @classmethod
+    def with_adapters(cls, desc: cql_desc, W, act_absmean=None, naive: bool = False, stream=None):
+        """Pack W with adapters built on the GPU from its own compression
+        error: SLiM-LoRA weighted by ``act_absmean`` (Naive-LoRA when
+        ``naive`` or when no statistic is given).  Packs with zero adapters,
+        builds L and R (cql_build_adapters), packs again with them.  The
+        built factors are kept as ``.L`` and ``.R``."""
+        import torch
+        dev = W.device
+        r = desc.rank
+        zL = torch.zeros(desc.n_out, r, dtype=torch.float32, device=dev)
+        zR = torch.zeros(r, desc.k_in, dtype=torch.float32, device=dev)
+        first = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean)
+        nb = cql_adapter_workspace_size(desc)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+        stat = None if (naive or act_absmean is None) else act_absmean.contiguous()
+        cql_build_adapters(desc, W.contiguous(), _dt_of(W), first.packed, stat, zL, zR, ws, nb, stream)
+        layer = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean)
+        layer.L, layer.R = zL, zR
+        layer._build_ws = (ws, first)            # alive until the queued kernels ran
+        return layer
 
     def workspace(self, batch: int, stream=None):
         import torch

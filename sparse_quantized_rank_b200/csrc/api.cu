@@ -87,6 +87,29 @@ HeaderBytes make_header(const cql_desc& d, const cql_layout& L) {
   return h;
 }
 
+// The layer's plane pointers and sizes, as every kernel reads them.
+DecodeParams planes_of(const cql_desc& d, const void* packed, const cql_layout& lay) {
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.d = d;
+  p.rb = row_bytes_of(d);
+  p.header = base;
+  p.values = base + lay.off[CQL_PLANE_VALUES];
+  p.meta = base + lay.off[CQL_PLANE_META];
+  p.scales = base + lay.off[CQL_PLANE_SCALES];
+  p.voff = base + lay.off[CQL_PLANE_VOFF];
+  p.csr_rowptr = d.outlier_frac > 0.0f ? reinterpret_cast<const int32_t*>(base + lay.off[CQL_PLANE_CSR_ROWPTR]) : nullptr;
+  p.csr_col = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_CSR_COL]);
+  p.csr_val = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_CSR_VAL]);
+  p.r_values = base + lay.off[CQL_PLANE_R_VALUES];
+  p.r_scales = base + lay.off[CQL_PLANE_R_SCALES];
+  p.l_values = base + lay.off[CQL_PLANE_L_VALUES];
+  p.l_scales = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_L_SCALES]);
+  p.nnz = lay.nnz;
+  return p;
+}
+
 int padded_batch(int b) {
   if (b <= 1) return 1;
   if (b <= 2) return 2;
@@ -271,23 +294,7 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   compute_layout(d, &lay);
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  DecodeParams p;
-  memset(&p, 0, sizeof(p));
-  p.d = d;
-  p.rb = row_bytes_of(d);
-  p.header = base;
-  p.values = base + lay.off[CQL_PLANE_VALUES];
-  p.meta = base + lay.off[CQL_PLANE_META];
-  p.scales = base + lay.off[CQL_PLANE_SCALES];
-  p.voff = base + lay.off[CQL_PLANE_VOFF];
-  p.csr_rowptr = d.outlier_frac > 0.0f ? reinterpret_cast<const int32_t*>(base + lay.off[CQL_PLANE_CSR_ROWPTR]) : nullptr;
-  p.csr_col = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_CSR_COL]);
-  p.csr_val = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_CSR_VAL]);
-  p.r_values = base + lay.off[CQL_PLANE_R_VALUES];
-  p.r_scales = base + lay.off[CQL_PLANE_R_SCALES];
-  p.l_values = base + lay.off[CQL_PLANE_L_VALUES];
-  p.l_scales = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_L_SCALES]);
-  p.nnz = lay.nnz;
+  DecodeParams p = planes_of(d, packed, lay);
   p.x = x;
   p.xdt = (int)x_dt;
   p.y = y;
@@ -314,6 +321,39 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   const cudaError_t e = batch > CQL_MAX_DECODE_BATCH
                             ? launch_prefill(p, ws + fw.prefill, reinterpret_cast<cudaStream_t>(stream))
                             : launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CQL_OK : CQL_ERR_CUDA;
+}
+
+cql_status cql_adapter_workspace_size(const cql_desc* desc, uint64_t* bytes) {
+  if (bytes == nullptr) return CQL_ERR_ARG;
+  const cql_status s = validate_desc(desc);
+  if (s != CQL_OK) return s;
+  if (desc->rank <= 0 || desc->rank > desc->n_out || desc->rank > desc->k_in) return CQL_ERR_ARG;
+  *bytes = lora_workspace_layout(*desc).total;
+  return CQL_OK;
+}
+
+cql_status cql_build_adapters(const cql_desc* desc, const void* W, cql_dtype w_dt, const void* packed,
+                              const float* act_absmean, float* L, float* R, void* workspace, uint64_t ws_bytes,
+                              cql_stream_t stream) {
+  uint64_t need = 0;
+  const cql_status s = cql_adapter_workspace_size(desc, &need);
+  if (s != CQL_OK) return s;
+  if (W == nullptr || packed == nullptr || L == nullptr || R == nullptr || workspace == nullptr) return CQL_ERR_ARG;
+  if (w_dt != CQL_DT_F32 && w_dt != CQL_DT_BF16) return CQL_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 256) || !aligned(workspace, 256) || !aligned(L, 4) || !aligned(R, 4) ||
+      (act_absmean != nullptr && !aligned(act_absmean, 4)))
+    return CQL_ERR_ALIGN;
+  if (ws_bytes < need) return CQL_ERR_SIZE;
+  cql_layout lay;
+  compute_layout(*desc, &lay);
+  const DecodeParams p = planes_of(*desc, packed, lay);
+  const uint16_t* sal = desc->salient_channels > 0
+                            ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(packed) +
+                                                                lay.off[CQL_PLANE_SALIENT])
+                            : nullptr;
+  const cudaError_t e = launch_build_adapters(p, W, (int)w_dt, act_absmean, sal, static_cast<uint8_t*>(workspace),
+                                              L, R, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CQL_OK : CQL_ERR_CUDA;
 }
 

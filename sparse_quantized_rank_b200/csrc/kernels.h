@@ -124,6 +124,17 @@ CQL_DEV bool header_ok(const DecodeParams& p) {
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
 
+// SLiM-LoRA / Naive-LoRA adapter construction (lora.cu).
+struct LoraWorkspace {
+  uint64_t es, y, y2, z, z2, g, u, ri, v, sig, ord, colf, xbarp, total;
+};
+int lora_width(const cql_desc& d);                     // subspace width p
+LoraWorkspace lora_workspace_layout(const cql_desc& d);
+// p: the layer's planes (as for a forward); act: mean |x_c| or null
+// (Naive-LoRA); salient: the SALIENT plane (SLiM^O) or null.
+cudaError_t launch_build_adapters(const DecodeParams& p, const void* W, int wdt, const float* act,
+                                  const uint16_t* salient, uint8_t* ws, float* L, float* R, cudaStream_t st);
+
 // SLiM^O forward prologue: xs = x with the listed channels divided by
 // 2^salient_log2 (same dtype, [batch][K]); PDL-chained to the kernel before.
 cudaError_t launch_salient_x(const DecodeParams& p, const uint16_t* list, void* xs, cudaStream_t st);
