@@ -15,8 +15,13 @@ Sources (web pages summarising the methods):
   adapter quantization" (AbsMax, groups of 128); rebuttal sections
   "Unstructured vs. 2:4 Sparsity" and "Order of Pruning and Quantization".
 * SqueezeLLM: Dense-and-Sparse Quantization -- "Approach" (non-uniform LUT
-  quantisation; the top 0.45% outliers go to a full-precision CSR matrix so
+  quantisation whose k-means centroids are weighted by a diagonal Fisher
+  information; the top 0.45% outliers go to a full-precision CSR matrix so
   the dense part has a narrower range).
+* SLiM review summary, "SLIM-Quant", and rebuttal, "Assumptions in
+  Theoretical Derivations": the clip threshold alpha is found by a grid
+  search over a probabilistic (histogram-based) model of the quantisation
+  error.
 * SLiM (same page), review summary "SLIM-LoRA" and rebuttal "Assumptions in
   Theoretical Derivations": the adapters minimise the saliency-weighted
   error norm ||F(W - W_C - L R)|| for an additive, invertible saliency F
@@ -61,6 +66,8 @@ __all__ = [
     "build_csr", "compress", "packed_layout", "pack_bytes",
     "channel_saliency", "select_salient_channels", "scale_activations",
     "compressed_matrix", "slim_lora", "lowrank_objective", "build_adapters",
+    "ALPHA_GRID", "ALPHA_BINS", "clip_histogram", "alpha_objective", "search_clip_alpha",
+    "KMEANS_MAX_ITERS", "fisher_kmeans",
     "forward", "forward_terms", "dense_reconstruction",
     "rel_err", "pack_and_forward", "HEADER_BYTES", "NPLANES",
     "P_HEADER", "P_VALUES", "P_META", "P_SCALES", "P_VOFF", "P_CSR_ROWPTR",
@@ -234,6 +241,58 @@ def quantize_uniform(w: np.ndarray, bits: int, alpha: float,
     return q, s
 
 
+ALPHA_GRID = tuple(i / 100 for i in range(30, 101))   # candidate clip thresholds 0.30 .. 1.00
+ALPHA_BINS = 1024
+
+
+def clip_histogram(w: np.ndarray, keep: np.ndarray, exclude: Optional[np.ndarray] = None) -> np.ndarray:
+    """Empirical distribution of the normalised magnitudes t = |w| / amax_g
+    (amax_g over the group's non-outlier entries, as the codec takes it) of
+    the entries the codec's error reaches: kept by the mask, not outliers, in
+    groups with amax_g > 0.  Bin b = min(floor((|w| / amax_g) * 1024), 1023),
+    evaluated in fp64.  Returns int64 counts [1024]."""
+    a = np.abs(np.asarray(w, dtype=np.float64))
+    n, k = a.shape
+    ae = np.where(exclude, 0.0, a) if exclude is not None else a
+    amax = np.repeat(ae.reshape(n, k // GROUP, GROUP).max(axis=2), GROUP, axis=1)
+    use = keep & (amax > 0)
+    if exclude is not None:
+        use &= ~exclude
+    with np.errstate(divide="ignore", invalid="ignore"):
+        b = np.floor((a / np.where(amax > 0, amax, 1.0)) * ALPHA_BINS)
+    b = np.minimum(b, ALPHA_BINS - 1).astype(np.int64)
+    return np.bincount(b[use], minlength=ALPHA_BINS).astype(np.int64)
+
+
+def alpha_objective(counts: np.ndarray, bits: int, alpha: float) -> float:
+    """Expected squared error (in units of amax^2, up to the entry count) of
+    symmetric clipped RTN with threshold alpha over the histogram: bin b
+    stands for its centre c_b = (b + 1/2) / 1024, quantised to
+    Q(c) = min(rint((c qmax) / alpha), qmax) * alpha / qmax; the sum
+    sum_b count_b (c_b - Q(c_b))^2 runs over b in order (fp64; alpha is the
+    fp32 value)."""
+    qmax = float((1 << (bits - 1)) - 1)
+    al = _f32(alpha)
+    c = (np.arange(ALPHA_BINS, dtype=np.float64) + 0.5) / ALPHA_BINS
+    q = np.minimum(np.rint((c * qmax) / al), qmax)
+    d = c - (q * al) / qmax
+    return float(np.cumsum(np.asarray(counts, dtype=np.float64) * (d * d))[-1])
+
+
+def search_clip_alpha(counts: np.ndarray, bits: int) -> float:
+    """SLiM-Quant's grid search: the candidate of ALPHA_GRID (as fp32) with
+    the least alpha_objective, ties to the smaller alpha.  Readings: the
+    pages give neither the grid nor the bin count; a layer-wide alpha (the
+    descriptor holds one) from a 1024-bin histogram of |w| / amax_g over
+    0.30 .. 1.00 in steps of 0.01."""
+    best, best_v = None, None
+    for a in ALPHA_GRID:
+        v = alpha_objective(counts, bits, a)
+        if best_v is None or v < best_v:
+            best, best_v = a, v
+    return float(np.float32(best))
+
+
 # ---------------------------------------------------------------------------
 # LUT codec: SqueezeLLM-style non-uniform per-row table
 # ---------------------------------------------------------------------------
@@ -270,6 +329,56 @@ def lut_centroids(w: np.ndarray, bits: int, exclude: Optional[np.ndarray] = None
         c = vlo + frac * (vhi - vlo)
         out[:, j] = np.where(nr > 0, c, 0.0) + 0.0      # -0 -> +0
     return fp16_round(out)
+
+
+KMEANS_MAX_ITERS = 32
+
+
+def fisher_kmeans(w: np.ndarray, cent0: np.ndarray, fisher: np.ndarray,
+                  exclude: Optional[np.ndarray] = None, max_iters: int = KMEANS_MAX_ITERS,
+                  round_fp16: bool = True) -> np.ndarray:
+    """Sensitivity-weighted k-means of every row (SqueezeLLM "Approach":
+    centroids weighted by the diagonal Fisher information).
+
+    Lloyd iterations from the initial table cent0 [N][2^b]: each non-outlier
+    value of the row goes to its nearest centroid (fp64 |v - c_j|, ties to the
+    lower j); each centroid becomes sum f v / sum f over its members (f the
+    fp32 Fisher diagonal; a centroid with no weight keeps its value).  A row
+    stops when an assignment repeats the previous one, or after max_iters
+    updates.  Readings: the initial table is the quantile table; sums run in
+    column order (sequentially, fp64, products f v exact); the result is
+    rounded to fp16 (+0 for a zero).  Returns fp64 [N][2^b] of fp16 values
+    (unrounded fp64 with round_fp16=False)."""
+    v = np.asarray(w, dtype=np.float64)
+    f = np.asarray(fisher, dtype=np.float32).astype(np.float64)
+    n, k = v.shape
+    c = np.array(cent0, dtype=np.float64, copy=True)
+    nc = c.shape[1]
+    member = np.ones((n, k), dtype=bool) if exclude is None else ~exclude
+    fv = f * v
+    prev = None
+    active = np.ones(n, dtype=bool)
+    for _ in range(max_iters):
+        best = np.abs(v - c[:, 0:1])
+        asg = np.zeros((n, k), dtype=np.int64)
+        for j in range(1, nc):
+            dj = np.abs(v - c[:, j:j + 1])
+            better = dj < best                           # strict: ties to the lower j
+            asg[better] = j
+            best = np.where(better, dj, best)
+        if prev is not None:
+            same = np.all((asg == prev) | ~member, axis=1)
+            active &= ~same
+        if not active.any():
+            break
+        for j in range(nc):
+            m = member & (asg == j)
+            num = np.cumsum(np.where(m, fv, 0.0), axis=1)[:, -1]
+            den = np.cumsum(np.where(m, f, 0.0), axis=1)[:, -1]
+            upd = active & (den > 0)
+            c[upd, j] = num[upd] / den[upd]
+        prev = asg
+    return fp16_round(c) + 0.0 if round_fp16 else c
 
 
 def lut_assign(w: np.ndarray, cent: np.ndarray) -> np.ndarray:
@@ -404,7 +513,8 @@ def scale_activations(x: np.ndarray, salient: np.ndarray, log2: int) -> np.ndarr
 # ---------------------------------------------------------------------------
 
 def compress(desc: OracleDesc, w: np.ndarray, L: Optional[np.ndarray] = None,
-             R: Optional[np.ndarray] = None, act_absmean: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+             R: Optional[np.ndarray] = None, act_absmean: Optional[np.ndarray] = None,
+             fisher: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Run the encoding steps in order: (SLiM^O) salient-channel scaling,
     outliers, mask, codec, CSR, adapters.
 
@@ -447,13 +557,19 @@ def compress(desc: OracleDesc, w: np.ndarray, L: Optional[np.ndarray] = None,
 
     bits = _CODEC_BITS[desc.codec]
     if desc.codec in (CODEC_INT4, CODEC_INT3):
-        q, s = quantize_uniform(w, bits, desc.clip_alpha, exclude=is_out if ns else None)
+        alpha = desc.clip_alpha
+        if alpha == 0:                                  # SLiM-Quant alpha search
+            alpha = search_clip_alpha(clip_histogram(w, keep, is_out if ns else None), bits)
+        parts["clip_alpha"] = np.float64(np.float32(alpha))
+        q, s = quantize_uniform(w, bits, alpha, exclude=is_out if ns else None)
         dense = np.where(keep, q.astype(np.float64) * np.repeat(s, GROUP, axis=1), 0.0)
         parts["q"] = q
         parts["scales"] = s
         parts["codes"] = (q.astype(np.int16) + (1 << (bits - 1))).astype(np.uint8)
     else:
         cent = lut_centroids(w, bits, exclude=is_out if ns else None)
+        if fisher is not None:                          # SqueezeLLM sensitivity-weighted k-means
+            cent = fisher_kmeans(w, cent, fisher, exclude=is_out if ns else None)
         code = lut_assign(w, cent)
         dense = np.where(keep, np.take_along_axis(cent, code.astype(np.int64), axis=1), 0.0)
         parts["centroids"] = cent
@@ -724,11 +840,11 @@ def _f16_bits(v: np.ndarray) -> np.ndarray:
     return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
 
 
-def _header(desc: OracleDesc, lay: dict) -> np.ndarray:
+def _header(desc: OracleDesc, lay: dict, alpha=None) -> np.ndarray:
     d = struct.pack(
         "<iiiiiffiiiIii12x",
         desc.n_out, desc.k_in, desc.mask, desc.codec, desc.group,
-        np.float32(desc.clip_alpha), np.float32(desc.outlier_frac), desc.rank,
+        np.float32(desc.clip_alpha if alpha is None else alpha), np.float32(desc.outlier_frac), desc.rank,
         desc.adapter_bits, desc.adapter_group, desc.flags, desc.salient_channels, desc.salient_log2)
     assert len(d) == 64
     body = b"CQL1" + struct.pack("<I", FORMAT_VERSION) + d
@@ -752,7 +868,7 @@ def pack_bytes(desc: OracleDesc, parts: Dict[str, np.ndarray]) -> np.ndarray:
         assert data.size == lay["len"][plane], (plane, data.size, lay["len"][plane])
         buf[lay["off"][plane]: lay["off"][plane] + data.size] = data
 
-    put(P_HEADER, _header(desc, lay))
+    put(P_HEADER, _header(desc, lay, parts.get("clip_alpha")))
     bits = _CODEC_BITS[desc.codec]
     keep = parts["keep"]
     codes = parts["codes"]
@@ -805,7 +921,7 @@ def pack_bytes(desc: OracleDesc, parts: Dict[str, np.ndarray]) -> np.ndarray:
     return buf
 
 
-def pack_and_forward(desc: OracleDesc, w, L, R, x, act_absmean=None):
+def pack_and_forward(desc: OracleDesc, w, L, R, x, act_absmean=None, fisher=None):
     """Convenience: (packed bytes, parts, y fp64)."""
-    parts = compress(desc, w, L, R, act_absmean)
+    parts = compress(desc, w, L, R, act_absmean, fisher)
     return pack_bytes(desc, parts), parts, forward(parts, x)

@@ -14,7 +14,10 @@ the same value structure the workload descriptions ask for:
 * for the output-error (SLiM^O) variant, a per-channel activation statistic
   mean|x_c| drawn as exp(0.5 N(0, 1)) with 0.5% of the channels multiplied by
   30 (the few "massive" activation channels LLMs show), from its own stream
-  (PCG64 seeded with (seed, 1)) so the other draws are unchanged.
+  (PCG64 seeded with (seed, 1)) so the other draws are unchanged;
+* for the sensitivity-weighted LUT (SqueezeLLM), a diagonal Fisher
+  information drawn as squared N(0, 1) gradients (chi-square, 1 degree of
+  freedom; heavy-tailed positive weights), stream (seed, 2).
 
 Every array is drawn from ``numpy.random.default_rng(seed)`` (PCG64) in a fixed
 order: W, the spike positions, L, R, x.  Nothing here masks, quantises or
@@ -91,6 +94,7 @@ class Workload:
     note: str = ""
     salient_channels: int = 0   # SLiM^O: channels scaled (0 = plain SLiM)
     salient_log2: int = 0       # SLiM^O: factor 2**salient_log2
+    fisher: bool = False        # draw a Fisher diagonal (LUT k-means weights)
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -186,7 +190,9 @@ def make_layer_inputs(wl: Workload, max_batch: Optional[int] = None) -> dict:
       ``x``      float32 [B][K], the exact delivered activation values,
       ``x_bits`` uint16 [B][K] (fp16 or bf16 patterns),
       ``act_absmean`` float32 [K] per-channel mean |x| statistic (SLiM^O
-                 workloads; None otherwise).
+                 workloads; None otherwise),
+      ``fisher`` float32 [N][K] Fisher diagonal (workloads with fisher=True;
+                 None otherwise).
     """
     rng = np.random.default_rng(wl.seed)
     n, k = wl.n, wl.k
@@ -214,7 +220,12 @@ def make_layer_inputs(wl: Workload, max_batch: Optional[int] = None) -> dict:
         heavy = arng.choice(k, size=max(1, k // 200), replace=False)
         a[heavy] *= 30.0
         act = a.astype(np.float32)
-    return {"w": w32, "w_bits": w_bits, "L": L, "R": R, "x": x32, "x_bits": x_bits, "act_absmean": act}
+    fis = None
+    if wl.fisher:
+        g = np.random.default_rng((wl.seed, 2)).standard_normal((n, k))
+        fis = (g * g).astype(np.float32)
+    return {"w": w32, "w_bits": w_bits, "L": L, "R": R, "x": x32, "x_bits": x_bits, "act_absmean": act,
+            "fisher": fis}
 
 
 def make_activations(k: int, batch: int, dtype: str, seed: int):
