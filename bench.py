@@ -216,7 +216,7 @@ def cpu_oracle_rate(wl, batch, seconds, steps=None, warmup=0):
     from workloads import make_layer_inputs
     inp = make_layer_inputs(wl, max_batch=batch)
     od = O.desc_for(wl)
-    parts = O.compress(od, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
+    parts = O.compress(od, inp["w"], inp["L"], inp["R"], inp["act_absmean"], inp["fisher"])
     lay = O.packed_layout(od)
     x = inp["x"][:batch].astype(np.float64)
     planes = sum(lay["len"][i] for i in range(len(lay["len"])) if i not in (O.P_HEADER, O.P_VOFF))
@@ -297,7 +297,8 @@ class Bench:
         W, L, R, x = device_inputs(torch, inp, wl, dev)
         self.desc = desc_from_workload(C, wl)
         act = None if inp["act_absmean"] is None else torch.from_numpy(inp["act_absmean"]).to(dev)
-        self.layer = C.CompressedLinear(self.desc, W, L, R, act_absmean=act)
+        fis = None if inp["fisher"] is None else torch.from_numpy(inp["fisher"]).to(dev)
+        self.layer = C.CompressedLinear(self.desc, W, L, R, act_absmean=act, fisher=fis)
         self.desc.flags = flags                     # forward-only flags (the packed header keeps 0)
         del W, L, R
         torch.cuda.synchronize()

@@ -110,9 +110,22 @@
  *   3. int codecs: s = fp16((alpha * amax) / qmax) with amax over the group's
  *      non-outlier entries, q = clamp(rint(w / s), -qmax, qmax), q = 0 when
  *      s = 0; qmax = 7 (int4) or 3 (int3);
+ *      clip_alpha = 0 (SLiM-Quant search): counts h_b, b < 1024, of
+ *      b = min(floor((|w| / amax) * 1024), 1023) over the kept non-outlier
+ *      entries of groups with amax > 0; for alpha_i = fp32(i / 100),
+ *      i = 30..100, E_i = sum_b h_b d_b^2 (b ascending, fp64, no fused
+ *      operations) with c = (b + 1/2) / 1024, q = min(rint((c qmax) /
+ *      alpha_i), qmax), d = c - (q alpha_i) / qmax; alpha = the alpha_i of
+ *      least E_i (ties to the smaller), written into the header's descriptor;
  *      lut codecs: centroid j = linear-interpolated quantile of the row's
- *      sorted non-outlier values at p = (j + 1/2)/2^b, rounded to fp16; every
- *      entry takes the nearest centroid;
+ *      sorted non-outlier values at p = (j + 1/2)/2^b, rounded to fp16; with
+ *      a Fisher diagonal f (SqueezeLLM sensitivity-weighted k-means) these
+ *      start Lloyd iterations instead: each non-outlier value goes to the
+ *      nearest centroid (fp64, ties to the lower), an assignment equal to
+ *      the previous one stops, else centroid j = (sum f v) / (sum f) over
+ *      its members in column order (a centroid without weight stays), at
+ *      most 32 updates, then rounded to fp16; every entry takes the nearest
+ *      centroid;
  *   4. CSR values as above;
  *   5. adapters: s = fp16(amax / 7), q = clamp(rint(v / s), -7, 7), groups of
  *      128 along K for R and along N for L.
@@ -179,7 +192,7 @@ typedef struct cql_desc {
   int32_t mask;           /* cql_mask                                        */
   int32_t codec;          /* cql_codec; lut codecs need CQL_MASK_NONE        */
   int32_t group;          /* weight scale group; must be 128                 */
-  float clip_alpha;       /* SLiM-Quant clip alpha in (0, 1]                 */
+  float clip_alpha;       /* SLiM-Quant clip alpha in (0, 1]; 0 = search it  */
   float outlier_frac;     /* CSR fraction f in [0, 1/16]; 0 = no CSR         */
   int32_t rank;           /* adapter rank r, multiple of 16, <= 256; 0 = none */
   int32_t adapter_bits;   /* must be 4                                       */
@@ -222,6 +235,9 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
  *   act_absmean  device fp32 [K], the mean |x_c| of each input channel over
  *             calibration tokens (finite, >= 0); required when
  *             salient_channels > 0, ignored (may be NULL) otherwise.
+ *   fisher    device fp32 [N][K] diagonal Fisher information (finite, >= 0)
+ *             for the LUT codecs' weighted k-means, or NULL (quantile
+ *             table); ignored by the int codecs.
  *   packed    device, >= cql_layout.total_bytes, 256-byte aligned; every byte
  *             of it is written.
  *   workspace device scratch of >= cql_pack_workspace_size bytes, 256-byte
@@ -229,7 +245,8 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
  * The result is bit-exact with the CPU oracle on every byte.  Inputs must be
  * finite. */
 cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt,
-                                  const float* L, const float* R, const float* act_absmean, void* packed,
+                                  const float* L, const float* R, const float* act_absmean,
+                                  const float* fisher, void* packed,
                                   uint64_t packed_bytes, void* workspace, uint64_t ws_bytes,
                                   cql_stream_t stream);
 

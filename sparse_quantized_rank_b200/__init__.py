@@ -80,8 +80,8 @@ def lib():
         L.cql_version.restype = I32
         L.cql_packed_layout.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(cql_layout)]
         L.cql_pack_workspace_size.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(U64)]
-        L.pack_compressed_weight.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, U64, P, U64,
-                                             P]
+        L.pack_compressed_weight.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, P, U64, P,
+                                             U64, P]
         L.cql_workspace_size.argtypes = [ctypes.POINTER(cql_desc), I32, ctypes.POINTER(U64)]
         L.cql_workspace_init.argtypes = [P, U64, P]
         L.compressed_linear_forward.argtypes = [ctypes.POINTER(cql_desc), P, P, ctypes.c_int, P, ctypes.c_int,
@@ -154,11 +154,11 @@ def cql_pack_workspace_size(desc: cql_desc) -> int:
     return int(v.value)
 
 
-def pack_compressed_weight(desc, W, w_dt, L, R, act_absmean, packed, packed_bytes, workspace, ws_bytes,
+def pack_compressed_weight(desc, W, w_dt, L, R, act_absmean, fisher, packed, packed_bytes, workspace, ws_bytes,
                            stream=None):
     _check(lib().pack_compressed_weight(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(L), _ptr(R), _ptr(act_absmean),
-                                        _ptr(packed), int(packed_bytes), _ptr(workspace), int(ws_bytes),
-                                        _stream(stream)),
+                                        _ptr(fisher), _ptr(packed), int(packed_bytes), _ptr(workspace),
+                                        int(ws_bytes), _stream(stream)),
            "pack_compressed_weight")
 
 
@@ -220,11 +220,13 @@ class CompressedLinear:
 
     ``W`` is a CUDA tensor [N][K] (fp32 or bf16), ``L`` [N][r] and ``R`` [r][K]
     fp32 CUDA tensors (or None when rank is 0), ``act_absmean`` a fp32 CUDA
-    tensor [K] of per-channel mean |x| (SLiM^O layers only).  Buffers are
-    torch tensors allocated once; forward calls allocate only the output
-    tensor (or write into ``out``)."""
+    tensor [K] of per-channel mean |x| (SLiM^O layers only), ``fisher`` a
+    fp32 CUDA tensor [N][K] Fisher diagonal (LUT codecs: weighted k-means).
+    A descriptor with clip_alpha 0 has the packer search alpha; the chosen
+    value is in ``clip_alpha()``.  Buffers are torch tensors allocated once;
+    forward calls allocate only the output tensor (or write into ``out``)."""
 
-    def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None, act_absmean=None):
+    def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None, act_absmean=None, fisher=None):
         import torch
         self.desc = desc
         self.layout = cql_packed_layout(desc)
@@ -234,13 +236,19 @@ class CompressedLinear:
         pws = torch.empty(max(pw, 256), dtype=torch.uint8, device=dev)
         pack_compressed_weight(desc, W.contiguous(), _dt_of(W), None if L is None else L.contiguous(),
                                None if R is None else R.contiguous(),
-                               None if act_absmean is None else act_absmean.contiguous(), self.packed,
+                               None if act_absmean is None else act_absmean.contiguous(),
+                               None if fisher is None else fisher.contiguous(), self.packed,
                                self.layout.total_bytes, pws, pw, stream)
         self._pack_ws = pws            # kept alive until the pack kernels ran
         self._ws = {}
 
+    def clip_alpha(self) -> float:
+        """The clip threshold the layer was encoded with (read from the packed
+        header: the searched value when the descriptor asked for a search)."""
+        return float(self.packed[28:32].cpu().view(__import__("torch").float32).item())
+
     @classmethod
-    def with_adapters(cls, desc: cql_desc, W, act_absmean=None, naive: bool = False, stream=None):
+    def with_adapters(cls, desc: cql_desc, W, act_absmean=None, naive: bool = False, stream=None, fisher=None):
         """Pack W with adapters built on the GPU from its own compression
         error: SLiM-LoRA weighted by ``act_absmean`` (Naive-LoRA when
         ``naive`` or when no statistic is given).  Packs with zero adapters,
@@ -251,12 +259,12 @@ class CompressedLinear:
         r = desc.rank
         zL = torch.zeros(desc.n_out, r, dtype=torch.float32, device=dev)
         zR = torch.zeros(r, desc.k_in, dtype=torch.float32, device=dev)
-        first = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean)
+        first = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean, fisher=fisher)
         nb = cql_adapter_workspace_size(desc)
         ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
         stat = None if (naive or act_absmean is None) else act_absmean.contiguous()
         cql_build_adapters(desc, W.contiguous(), _dt_of(W), first.packed, stat, zL, zR, ws, nb, stream)
-        layer = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean)
+        layer = cls(desc, W, zL, zR, stream=stream, act_absmean=act_absmean, fisher=fisher)
         layer.L, layer.R = zL, zR
         layer._build_ws = (ws, first)            # alive until the queued kernels ran
         return layer

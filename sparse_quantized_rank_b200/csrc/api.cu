@@ -19,7 +19,7 @@ cql_status validate_desc(const cql_desc* d) {
   if (d->mask < CQL_MASK_NONE || d->mask > CQL_MASK_BITMAP50) return CQL_ERR_ARG;
   if (d->codec < CQL_CODEC_INT4_SYM || d->codec > CQL_CODEC_LUT4_ROW) return CQL_ERR_ARG;
   if (d->group != 128 || d->adapter_bits != 4 || d->adapter_group != 128) return CQL_ERR_UNSUPPORTED;
-  if (!(d->clip_alpha > 0.0f && d->clip_alpha <= 1.0f)) return CQL_ERR_ARG;
+  if (!(d->clip_alpha >= 0.0f && d->clip_alpha <= 1.0f)) return CQL_ERR_ARG;   // 0: search it
   if (!(d->outlier_frac >= 0.0f && d->outlier_frac <= 0.0625f)) return CQL_ERR_ARG;
   if (d->rank < 0 || d->rank > 256 || d->rank % 16 != 0) return CQL_ERR_ARG;
   if (d->salient_channels < 0 || d->salient_channels > d->k_in / 8) return CQL_ERR_ARG;
@@ -138,6 +138,7 @@ PackWorkspace pack_workspace_layout(const cql_desc& d) {
   w.sal_partial = pos; pos = align256(pos + (sal ? (uint64_t)(d.n_out / 64) * d.k_in * 8 : 0));
   w.sal = pos;       pos = align256(pos + (sal ? (uint64_t)d.k_in * 8 : 0));
   w.sal_flag = pos;  pos = align256(pos + (sal ? (uint64_t)d.k_in : 0));
+  w.alpha = pos;     pos = align256(pos + 1024 * 8 + 16);    // alpha histogram, then the alpha
   w.total = pos;
   return w;
 }
@@ -199,7 +200,7 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes) {
 }
 
 cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt, const float* L,
-                                  const float* R, const float* act_absmean, void* packed, uint64_t packed_bytes, void* workspace,
+                                  const float* R, const float* act_absmean, const float* fisher, void* packed, uint64_t packed_bytes, void* workspace,
                                   uint64_t ws_bytes, cql_stream_t stream) {
   cql_status s = validate_desc(desc);
   if (s != CQL_OK) return s;
@@ -211,6 +212,7 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
   if (d.rank > 0 && (!aligned(L, 16) || !aligned(R, 16))) return CQL_ERR_ALIGN;
   if (d.salient_channels > 0 && act_absmean == nullptr) return CQL_ERR_ARG;
   if (d.salient_channels > 0 && !aligned(act_absmean, 4)) return CQL_ERR_ALIGN;
+  if (fisher != nullptr && !aligned(fisher, 4)) return CQL_ERR_ALIGN;
   cql_layout lay;
   compute_layout(d, &lay);
   if (packed_bytes < lay.total_bytes) return CQL_ERR_SIZE;
@@ -253,6 +255,10 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
   p.sal_partial = reinterpret_cast<double*>(ws + pw.sal_partial);
   p.sal = reinterpret_cast<double*>(ws + pw.sal);
   p.sal_flag = ws + pw.sal_flag;
+  p.alpha_hist = reinterpret_cast<unsigned long long*>(ws + pw.alpha);
+  p.alpha_dev = (d.clip_alpha == 0.0f && !codec_is_lut(d.codec)) ? reinterpret_cast<float*>(ws + pw.alpha + 1024 * 8)
+                                                                : nullptr;
+  p.fisher = codec_is_lut(d.codec) ? fisher : nullptr;
   if (d.outlier_frac <= 0.0f) p.csr_rowptr = nullptr;
   const HeaderBytes h = make_header(d, lay);
   const cudaError_t e = launch_pack(p, h, lay.total_bytes, reinterpret_cast<cudaStream_t>(stream));

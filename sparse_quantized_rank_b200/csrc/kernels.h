@@ -54,10 +54,14 @@ struct PackParams {
   double* sal_partial;               // [N/64][K]
   double* sal;                       // [K]
   uint8_t* sal_flag;                 // [K]
+  // SLiM-Quant alpha search (clip_alpha 0) and SqueezeLLM Fisher k-means
+  float* alpha_dev;                  // the searched alpha (device), or null: use 'alpha'
+  unsigned long long* alpha_hist;    // [1024] histogram
+  const float* fisher;               // [N*K] Fisher diagonal (LUT codecs), or null
 };
 
 struct PackWorkspace {
-  uint64_t out_bits, state, hist, tiecnt, tieoff, row_counts, w_scaled, sal_partial, sal, sal_flag, total;
+  uint64_t out_bits, state, hist, tiecnt, tieoff, row_counts, w_scaled, sal_partial, sal, sal_flag, alpha, total;
 };
 PackWorkspace pack_workspace_layout(const cql_desc& d);
 

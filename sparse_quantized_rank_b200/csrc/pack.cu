@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
   const int n = blockIdx.x, K = p.d.k_in, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   constexpr int qmax = (1 << (BITS - 1)) - 1;
   const bool has_csr = p.out_bits != nullptr;
+  const double alpha = p.alpha_dev != nullptr ? (double)*p.alpha_dev : p.alpha;   // searched or given
   uint32_t kept_run = 0, out_run = has_csr ? (uint32_t)p.csr_rowptr[n] : 0u;
   for (int g = 0; g < K / kGroup; ++g) {
     const int c = g * kGroup + t;
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
     if (lane == 0) s_wmax[warp] = a;
     __syncthreads();
     const float amax = fmaxf(fmaxf(s_wmax[0], s_wmax[1]), fmaxf(s_wmax[2], s_wmax[3]));
-    const uint16_t s16 = f64_to_f16_bits(__ddiv_rn(__dmul_rn(p.alpha, (double)amax), (double)qmax));
+    const uint16_t s16 = f64_to_f16_bits(__ddiv_rn(__dmul_rn(alpha, (double)amax), (double)qmax));
     const double s = f16_to_f64(s16);
     const int q = rtn_code((double)wv, s, qmax);
     // kept index in the row stream
@@ -338,6 +339,89 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
     const uint32_t rbm = p.rb.meta;
     for (uint32_t j = t; j < rbm; j += 128)
       p.meta[rit(n, j, rbm)] = (uint8_t)((nib[2 * j] & 15u) | ((nib[2 * j + 1] & 15u) << 4));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// SLiM-Quant clip search (SLiM review summary, "SLIM-Quant"): histogram of
+// |w| / amax_g over the entries the codec's error reaches (kept by the mask,
+// not outliers), then the expected squared error of clipped RTN at the bin
+// centres for every candidate alpha; the least one (ties to the smaller) is
+// the layer's alpha.  Bin index and objective follow the format's rule
+// operation by operation in fp64 (no contraction), so the choice is
+// bit-exact.
+// ---------------------------------------------------------------------------
+constexpr int kAlphaBins = 1024;
+constexpr int kAlphaFirst = 30, kAlphaLast = 100;    // candidates i / 100
+
+template <int MASK>
+__global__ void __launch_bounds__(128) k_alpha_hist(PackParams p, unsigned long long* hist) {
+  __shared__ uint32_t h[kAlphaBins];
+  __shared__ float s_wmax[4];
+  const int n = blockIdx.x, K = p.d.k_in, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  for (int b = t; b < kAlphaBins; b += 128) h[b] = 0;
+  for (int g = 0; g < K / kGroup; ++g) {
+    const int c = g * kGroup + t;
+    const uint64_t idx = (uint64_t)n * K + c;
+    const float wv = wval(p.W, p.wdt, idx);
+    const uint32_t key = __float_as_uint(wv) & 0x7FFFFFFFu;
+    const bool outl = outlier_bit(p.out_bits, idx);
+    bool keep = true;
+    if (MASK == CQL_MASK_2_4) {
+      const int q0 = lane & ~3, i = lane & 3;
+      int rank = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t kj = __shfl_sync(0xffffffffu, key, q0 + j);
+        rank += (kj > key) || (kj == key && j < i);
+      }
+      keep = rank < 2;
+    } else if (MASK == CQL_MASK_BITMAP50) {
+      keep = (p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u;
+    }
+    float a = outl ? 0.0f : fabsf(wv);
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0) s_wmax[warp] = a;
+    __syncthreads();
+    const float amax = fmaxf(fmaxf(s_wmax[0], s_wmax[1]), fmaxf(s_wmax[2], s_wmax[3]));
+    if (keep && !outl && amax > 0.0f) {
+      const double b = floor(__dmul_rn(__ddiv_rn((double)fabsf(wv), (double)amax), (double)kAlphaBins));
+      atomicAdd(&h[b < kAlphaBins - 1 ? (int)b : kAlphaBins - 1], 1u);
+    }
+    __syncthreads();
+  }
+  for (int b = t; b < kAlphaBins; b += 128)
+    if (h[b]) atomicAdd(&hist[b], (unsigned long long)h[b]);
+}
+
+// one block: thread i evaluates candidate kAlphaFirst + i over the bins in
+// order; thread 0 picks the least, writes it to *alpha and into the packed
+// header's descriptor copy (clip_alpha at header byte 28)
+__global__ void __launch_bounds__(128) k_alpha_search(const unsigned long long* hist, int bits, float* alpha,
+                                                      uint8_t* packed) {
+  __shared__ double obj[128];
+  const int t = threadIdx.x;
+  const int ncand = kAlphaLast - kAlphaFirst + 1;
+  const double qmax = (double)((1 << (bits - 1)) - 1);
+  if (t < ncand) {
+    const double al = (double)__double2float_rn(__ddiv_rn((double)(kAlphaFirst + t), 100.0));
+    double s = 0.0;
+    for (int b = 0; b < kAlphaBins; ++b) {
+      const double c = __ddiv_rn(__dadd_rn((double)b, 0.5), (double)kAlphaBins);
+      const double q = fmin(rint(__ddiv_rn(__dmul_rn(c, qmax), al)), qmax);
+      const double d = __dsub_rn(c, __ddiv_rn(__dmul_rn(q, al), qmax));
+      s = __dadd_rn(s, __dmul_rn((double)hist[b], __dmul_rn(d, d)));
+    }
+    obj[t] = s;
+  }
+  __syncthreads();
+  if (t == 0) {
+    int best = 0;
+    for (int i = 1; i < ncand; ++i)
+      if (obj[i] < obj[best]) best = i;
+    const float a = __double2float_rn(__ddiv_rn((double)(kAlphaFirst + best), 100.0));
+    *alpha = a;
+    *reinterpret_cast<float*>(packed + 28) = a;
   }
 }
 
@@ -401,9 +485,53 @@ __global__ void __launch_bounds__(256, 1) k_codec_lut(PackParams p) {
     c = __dadd_rn(c, 0.0);                                    // -0 -> +0
     const uint16_t b = f64_to_f16_bits(c);
     cent[t] = f16_to_f64(b);
-    *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
+    if (p.fisher == nullptr) *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
   }
   __syncthreads();
+  if (p.fisher != nullptr) {
+    // SqueezeLLM sensitivity-weighted k-means (Lloyd, from the quantile
+    // table): assign every non-outlier value to its nearest centroid (ties to
+    // the lower), stop when an assignment repeats, else move each centroid to
+    // sum f v / sum f over its members, summed in column order; at most
+    // KMEANS iterations; round to fp16 at the end.
+    constexpr int kMaxIters = 32;
+    uint8_t* prev = codes + K;                                // K more bytes
+    for (int it = 0; it < kMaxIters; ++it) {
+      bool changed = false;
+      for (int c = t; c < K; c += 256) {
+        if (outlier_bit(p.out_bits, base + c)) continue;
+        const double wv = (double)wval(p.W, p.wdt, base + c);
+        uint32_t code = 0;
+        double best = fabs(__dsub_rn(wv, cent[0]));
+#pragma unroll
+        for (int j = 1; j < NC; ++j) {
+          const double d = fabs(__dsub_rn(wv, cent[j]));
+          if (d < best) { best = d; code = j; }
+        }
+        if (it > 0 && prev[c] != code) changed = true;
+        prev[c] = (uint8_t)code;
+      }
+      if (it > 0 && !__syncthreads_or(changed)) break;
+      __syncthreads();
+      if (t < NC) {
+        double num = 0.0, den = 0.0;
+        for (int c = 0; c < K; ++c) {
+          if (prev[c] != t || outlier_bit(p.out_bits, base + c)) continue;
+          const double f = (double)p.fisher[base + c];
+          num = __dadd_rn(num, __dmul_rn(f, (double)wval(p.W, p.wdt, base + c)));
+          den = __dadd_rn(den, f);
+        }
+        if (den > 0.0) cent[t] = __ddiv_rn(num, den);
+      }
+      __syncthreads();
+    }
+    if (t < NC) {
+      const uint16_t b = f64_to_f16_bits(__dadd_rn(cent[t], 0.0));
+      cent[t] = f16_to_f64(b);
+      *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
+    }
+    __syncthreads();
+  }
   const bool has_csr = p.out_bits != nullptr;
   uint32_t out_run = has_csr ? (uint32_t)p.csr_rowptr[n] : 0u;
   for (int chunk = 0; chunk < K; chunk += 256) {
@@ -525,7 +653,7 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
   if (codec_is_lut(p.d.codec)) {
     int P = 1;
     while (P < K) P <<= 1;
-    const size_t smem = (size_t)P * 4 + K;
+    const size_t smem = (size_t)P * 4 + K + (p.fisher != nullptr ? K : 0);
     if (p.d.codec == CQL_CODEC_LUT3_ROW) {
       if ((e = set_smem((const void*)k_codec_lut<3>, smem)) != cudaSuccess) return e;
       k_codec_lut<3><<<N, 256, smem, st>>>(p);
@@ -534,6 +662,14 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
       k_codec_lut<4><<<N, 256, smem, st>>>(p);
     }
   } else {
+    if (p.alpha_dev != nullptr) {                             // clip_alpha 0: search it
+      if ((e = cudaMemsetAsync(p.alpha_hist, 0, kAlphaBins * sizeof(unsigned long long), st)) != cudaSuccess)
+        return e;
+      if (p.d.mask == CQL_MASK_2_4) k_alpha_hist<CQL_MASK_2_4><<<N, 128, 0, st>>>(p, p.alpha_hist);
+      else if (p.d.mask == CQL_MASK_BITMAP50) k_alpha_hist<CQL_MASK_BITMAP50><<<N, 128, 0, st>>>(p, p.alpha_hist);
+      else k_alpha_hist<CQL_MASK_NONE><<<N, 128, 0, st>>>(p, p.alpha_hist);
+      k_alpha_search<<<1, 128, 0, st>>>(p.alpha_hist, codec_bits(p.d.codec), p.alpha_dev, p.packed);
+    }
     const size_t smem = (size_t)K + K / 4;
 #define CQL_LAUNCH_UNI(B, M)                                                   \
   do {                                                                         \

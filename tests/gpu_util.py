@@ -37,12 +37,16 @@ class Case:
         self.wl = wl
         self.inp = make_layer_inputs(wl, max_batch=max_batch)
         self.od = O.desc_for(wl)
-        self.parts = O.compress(self.od, self.inp["w"], self.inp["L"], self.inp["R"], self.inp["act_absmean"])
+        self.parts = O.compress(self.od, self.inp["w"], self.inp["L"], self.inp["R"], self.inp["act_absmean"],
+                                self.inp["fisher"])
         self.ref_bytes = O.pack_bytes(self.od, self.parts)
         self.W, self.L, self.R, self.x = device_inputs(self.inp, wl, dev)
         act = self.inp["act_absmean"]
         self.act = None if act is None else torch.from_numpy(act).to(dev)
-        self.layer = C.CompressedLinear(c_desc(self.od), self.W, self.L, self.R, act_absmean=self.act)
+        fis = self.inp["fisher"]
+        self.fisher = None if fis is None else torch.from_numpy(fis).to(dev)
+        self.layer = C.CompressedLinear(c_desc(self.od), self.W, self.L, self.R, act_absmean=self.act,
+                                        fisher=self.fisher)
         torch.cuda.synchronize()
 
     def packed_bytes(self):

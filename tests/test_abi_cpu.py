@@ -79,7 +79,7 @@ def test_descriptor_validation(lib):
         (dict(ok, codec=7), C.CQL_ERR_ARG),
         (dict(ok, rank=8), C.CQL_ERR_ARG),
         (dict(ok, rank=512), C.CQL_ERR_ARG),
-        (dict(ok, clip_alpha=0.0), C.CQL_ERR_ARG),
+        (dict(ok, clip_alpha=-0.1), C.CQL_ERR_ARG),
         (dict(ok, clip_alpha=1.5), C.CQL_ERR_ARG),
         (dict(ok, outlier_frac=-0.1), C.CQL_ERR_ARG),
         (dict(ok, codec=2), C.CQL_ERR_UNSUPPORTED),          # LUT needs no mask
@@ -121,19 +121,19 @@ def test_call_errors_return_before_launch(lib):
     st = L.compressed_linear_forward(ctypes.byref(d), fake, fake, C.CQL_DT_F16, fake, C.CQL_DT_F16, 0, fake, ws, None)
     assert st == C.CQL_ERR_ARG
     pw = C.cql_pack_workspace_size(d)
-    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, None, None, None, fake, lay.total_bytes, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, None, None, None, None, fake, lay.total_bytes, fake, pw,
                                   None)
     assert st == C.CQL_ERR_ARG                       # rank 16 needs L and R
-    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, fake, fake, None, fake, lay.total_bytes - 1, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake, C.CQL_DT_F32, fake, fake, None, None, fake, lay.total_bytes - 1, fake, pw,
                                   None)
     assert st == C.CQL_ERR_SIZE
-    st = L.pack_compressed_weight(ctypes.byref(d), fake + 8, C.CQL_DT_F32, fake, fake, None, fake, lay.total_bytes, fake, pw,
+    st = L.pack_compressed_weight(ctypes.byref(d), fake + 8, C.CQL_DT_F32, fake, fake, None, None, fake, lay.total_bytes, fake, pw,
                                   None)
     assert st == C.CQL_ERR_ALIGN
     ds = C.make_desc(256, 512, rank=16, salient_channels=5, salient_log2=1)
     lay_s = C.cql_packed_layout(ds)
     pws = C.cql_pack_workspace_size(ds)
-    st = L.pack_compressed_weight(ctypes.byref(ds), fake, C.CQL_DT_F32, fake, fake, None, fake, lay_s.total_bytes,
+    st = L.pack_compressed_weight(ctypes.byref(ds), fake, C.CQL_DT_F32, fake, fake, None, None, fake, lay_s.total_bytes,
                                   fake, pws, None)
     assert st == C.CQL_ERR_ARG                       # SLiM^O needs the activation statistic
     assert L.cql_get_device_status(None, None, None) == C.CQL_ERR_ARG
