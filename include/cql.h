@@ -153,7 +153,9 @@ typedef enum {
   CQL_ERR_SIZE = 4,         /* buffer or workspace too small                */
   CQL_ERR_UNSUPPORTED = 5,  /* valid but not implemented combination        */
   CQL_ERR_CUDA = 6,         /* a CUDA runtime call failed                   */
-  CQL_ERR_TIMEOUT = 7       /* a bounded device wait ran out                */
+  CQL_ERR_TIMEOUT = 7,      /* a bounded device wait ran out                */
+  CQL_ERR_RANGE = 8         /* checked build only: an index fell outside its
+                               buffer; the access was skipped (detail = site) */
 } cql_status;
 
 typedef enum { CQL_MASK_NONE = 0, CQL_MASK_2_4 = 1, CQL_MASK_BITMAP50 = 2 } cql_mask;

@@ -19,10 +19,11 @@ from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libcql.so")
+LIB_CHECKED_PATH = os.path.join(HERE, "libcql_checked.so")   # the range-checked build
 
 # enums (include/cql.h)
 CQL_OK, CQL_ERR_ARG, CQL_ERR_ALIGN, CQL_ERR_FORMAT, CQL_ERR_SIZE, CQL_ERR_UNSUPPORTED, \
-    CQL_ERR_CUDA, CQL_ERR_TIMEOUT = range(8)
+    CQL_ERR_CUDA, CQL_ERR_TIMEOUT, CQL_ERR_RANGE = range(9)
 CQL_MASK_NONE, CQL_MASK_2_4, CQL_MASK_BITMAP50 = 0, 1, 2
 CQL_CODEC_INT4_SYM, CQL_CODEC_INT3_SYM, CQL_CODEC_LUT3_ROW, CQL_CODEC_LUT4_ROW = 0, 1, 2, 3
 CQL_DT_F32, CQL_DT_F16, CQL_DT_BF16 = 0, 1, 2
@@ -63,17 +64,27 @@ class CqlError(RuntimeError):
         self.status = status
 
 
-_lib = None
+_libs = {}
+_active = LIB_PATH
+
+
+def use_library(checked: bool) -> None:
+    """Route every call of this module to the range-checked library
+    (libcql_checked.so, built with -DCQL_CHECKED) or back to libcql.so.
+    Objects keep the buffers they made with either; both libraries share the
+    packed format and the workspace layout."""
+    global _active
+    _active = LIB_CHECKED_PATH if checked else LIB_PATH
 
 
 def lib():
-    """The loaded libcql.so (raises if it is missing: there is no fallback)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m sparse_quantized_rank_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+    """The loaded library (raises if it is missing: there is no fallback)."""
+    if _active not in _libs:
+        if not os.path.exists(_active):
+            raise RuntimeError(f"{_active} is missing: build it with "
+                               "`python -m sparse_quantized_rank_b200.build`"
+                               + (" --checked" if _active == LIB_CHECKED_PATH else ""))
+        L = ctypes.CDLL(_active)
         P, U64, I32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int32
         L.cql_status_string.restype = ctypes.c_char_p
         L.cql_status_string.argtypes = [ctypes.c_int]
@@ -93,8 +104,8 @@ def lib():
         L.cql_build_adapters.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, P, U64, P]
         for fn in EXPORTED[2:]:
             getattr(L, fn).restype = ctypes.c_int
-        _lib = L
-    return _lib
+        _libs[_active] = L
+    return _libs[_active]
 
 
 def _ptr(t) -> Optional[int]:

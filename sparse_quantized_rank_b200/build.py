@@ -2,6 +2,13 @@
 
     python -m sparse_quantized_rank_b200.build          # build if stale
     python -m sparse_quantized_rank_b200.build --force  # always rebuild
+    python -m sparse_quantized_rank_b200.build --checked  # libcql_checked.so
+
+The checked variant is compiled with -DCQL_CHECKED: every plane read,
+activation read, workspace access and output store of the forward kernels
+is range-checked, and an index outside its buffer records CQL_ERR_RANGE in
+the device error word (the access is skipped) instead of touching memory.
+It stands in for a memory checker on machines where none can run.
 
 The library is compiled straight from ``csrc/*.cu`` with
 ``-gencode arch=compute_100a,code=sm_100a`` (B200 only) and the CUDA runtime
@@ -20,6 +27,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libcql.so")
+LIB_CHECKED = os.path.join(HERE, "libcql_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -40,26 +48,29 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source into libcql.so next to this file; return its path."""
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile every CUDA source into libcql.so (libcql_checked.so with
+    checked=True) next to this file; return its path."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = _nvcc()
-    objdir = os.path.join(HERE, "_build")
+    objdir = os.path.join(HERE, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
+    extra = ["-DCQL_CHECKED"] if checked else []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-dc" if False else "-c", src, "-o", obj]
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
@@ -69,19 +80,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if verbose and r.stderr:
             print(r.stderr, file=sys.stderr)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
            "-cudart", "static", *objs, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true", help="the range-checked variant")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, checked=a.checked))

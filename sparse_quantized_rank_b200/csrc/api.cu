@@ -107,6 +107,7 @@ DecodeParams planes_of(const cql_desc& d, const void* packed, const cql_layout& 
   p.l_values = base + lay.off[CQL_PLANE_L_VALUES];
   p.l_scales = reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_L_SCALES]);
   p.nnz = lay.nnz;
+  for (int i = 0; i < CQL_NPLANES; ++i) p.plane_len[i] = lay.len[i];
   return p;
 }
 
@@ -177,6 +178,7 @@ const char* cql_status_string(cql_status s) {
     case CQL_ERR_UNSUPPORTED: return "CQL_ERR_UNSUPPORTED: combination not implemented";
     case CQL_ERR_CUDA: return "CQL_ERR_CUDA: CUDA runtime error";
     case CQL_ERR_TIMEOUT: return "CQL_ERR_TIMEOUT: bounded device wait ran out";
+    case CQL_ERR_RANGE: return "CQL_ERR_RANGE: an index outside its buffer (checked build)";
   }
   return "CQL_ERR_UNKNOWN";
 }
@@ -317,6 +319,10 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
   p.counters = reinterpret_cast<uint32_t*>(ws + fw.counters);
   p.t_part = reinterpret_cast<float*>(ws + fw.t_part);
   p.t_final = reinterpret_cast<float*>(ws + fw.t_final);
+  p.x_elems = (uint64_t)batch * d.k_in;
+  p.y_elems = (uint64_t)batch * d.n_out;
+  p.t_final_elems = (fw.xs - fw.t_final) / 4;
+  p.t_part_elems = (fw.t_final - fw.t_part) / 4;
   if (d.salient_channels > 0) {
     // SLiM^O: every later step reads x' from the workspace
     const cudaError_t e0 = launch_salient_x(p, reinterpret_cast<const uint16_t*>(base + lay.off[CQL_PLANE_SALIENT]),

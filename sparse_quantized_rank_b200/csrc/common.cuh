@@ -65,6 +65,22 @@ CQL_DEV void set_error(uint32_t* err, uint32_t status, uint32_t detail) {
   if (atomicCAS(err, 0u, status) == 0u) atomicExch(err + 1, detail);
 }
 
+// Range checks of the checked build (compiled with -DCQL_CHECKED, the
+// library's stand-in for a memory checker): CQL_IN(err, i, n, site) is true
+// when 0 <= i < n; otherwise it records CQL_ERR_RANGE with the site number
+// as the detail and the caller skips the access.  In the normal build it is
+// the constant true and costs nothing.
+CQL_DEV bool in_range(uint32_t* err, uint64_t i, uint64_t n, uint32_t site) {
+  if (i < n) return true;
+  set_error(err, CQL_ERR_RANGE, site);
+  return false;
+}
+#ifdef CQL_CHECKED
+#define CQL_IN(err, i, n, site) ::cql::in_range((err), (uint64_t)(i), (uint64_t)(n), (site))
+#else
+#define CQL_IN(err, i, n, site) true
+#endif
+
 // ---------------------------------------------------------------------------
 // exact conversions
 // ---------------------------------------------------------------------------

@@ -42,7 +42,9 @@ constexpr int kEpiThreads = 128;                // epilogue block: four row bloc
 constexpr uint32_t kMagic = 0x4B000000u;       // fp32 bit pattern of 2^23
 
 CQL_DEV float act(const DecodeParams& p, int b, int col) {
-  return b < p.batch ? to_f32_act(p.x, p.xdt, (uint64_t)b * p.d.k_in + col) : 0.0f;
+  return b < p.batch && CQL_IN(p.err, (uint64_t)b * p.d.k_in + col, p.x_elems, 201)
+             ? to_f32_act(p.x, p.xdt, (uint64_t)b * p.d.k_in + col)
+             : 0.0f;
 }
 
 CQL_DEV uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
@@ -57,7 +59,8 @@ CQL_DEV void stage_x(const DecodeParams& p, float* xs, int c0, int ncols) {
   for (int i = threadIdx.x; i < B * chunks; i += blockDim.x) {
     const int b = i / chunks, ch = i - b * chunks;
     uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (b < p.batch) w = *reinterpret_cast<const uint4*>(xb + (uint64_t)b * p.d.k_in + c0 + 8 * ch);
+    if (b < p.batch && CQL_IN(p.err, (uint64_t)b * p.d.k_in + c0 + 8 * ch + 7, p.x_elems, 202))
+      w = *reinterpret_cast<const uint4*>(xb + (uint64_t)b * p.d.k_in + c0 + 8 * ch);
     const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -73,7 +76,8 @@ CQL_DEV void red_rows(const DecodeParams& p, int rb, const float (&acc)[B], int 
   const int row = rb * 32 + lane;
 #pragma unroll
   for (int b = 0; b < B; ++b)
-    if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
+    if (b < p.batch && CQL_IN(p.err, (uint64_t)b * p.d.n_out + row, p.y_elems, 203))
+      atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
 }
 
 // ---------------------------------------------------------------------------
@@ -145,11 +149,14 @@ struct Unit24 {
   static constexpr int kSlabs = 3;
   static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
     const uint32_t vs = BITS == 4 ? 2u * uk : (24u * uk) >> 4;
-    const uint8_t* vb = p.values + slab_off32(rb, vs, p.rb.values) + lane * 16;
-    cp_async16(slot, vb);
-    cp_async16(slot + 512, vb + 512);
-    cp_async16(slot + 1024, p.meta + slab_off32(rb, uk, p.rb.meta) + lane * 16);
-    const uint32_t sc = ldg_u16(p.scales + rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+    const uint32_t ov = slab_off32(rb, vs, p.rb.values) + lane * 16, om = slab_off32(rb, uk, p.rb.meta) + lane * 16;
+    const uint32_t os = rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales);
+    if (CQL_IN(p.err, ov + 512 + 15, p.plane_len[CQL_PLANE_VALUES], 204)) {
+      cp_async16(slot, p.values + ov);
+      cp_async16(slot + 512, p.values + ov + 512);
+    }
+    if (CQL_IN(p.err, om + 15, p.plane_len[CQL_PLANE_META], 205)) cp_async16(slot + 1024, p.meta + om);
+    const uint32_t sc = CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_SCALES], 206) ? ldg_u16(p.scales + os) : 0u;
     return sc | (BITS == 3 && ((24u * uk) & 15u) ? 0x10000u : 0u);
   }
   static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
@@ -253,15 +260,22 @@ struct UnitDense {
     float* lut = lut_base(smem, p) + (threadIdx.x >> 5) * (16 * 32);
     const uint64_t row = (uint64_t)rb * 32 + lane;
 #pragma unroll
-    for (int c = 0; c < (1 << BITS); ++c) lut[c * 32 + lane] = f16_bits_to_f32(ldg_u16(p.scales + rit(row, 2 * c, p.rb.scales)));
+    for (int c = 0; c < (1 << BITS); ++c)
+      lut[c * 32 + lane] = CQL_IN(p.err, rit(row, 2 * c, p.rb.scales) + 1, p.plane_len[CQL_PLANE_SCALES], 207)
+                               ? f16_bits_to_f32(ldg_u16(p.scales + rit(row, 2 * c, p.rb.scales)))
+                               : 0.0f;
     __syncwarp();
   }
   static constexpr int kSlabs = BITS;                     // 64 or 48 bytes of codes per unit
   static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
-    const uint8_t* vb = p.values + slab_off32(rb, (uint32_t)BITS * uk, p.rb.values) + lane * 16;
+    const uint32_t ov = slab_off32(rb, (uint32_t)BITS * uk, p.rb.values) + lane * 16;
+    if (CQL_IN(p.err, ov + 512 * (BITS - 1) + 15, p.plane_len[CQL_PLANE_VALUES], 208)) {
 #pragma unroll
-    for (int s = 0; s < BITS; ++s) cp_async16(slot + 512 * s, vb + 512 * s);
-    return LUT ? 0u : ldg_u16(p.scales + rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales));
+      for (int s = 0; s < BITS; ++s) cp_async16(slot + 512 * s, p.values + ov + 512 * s);
+    }
+    if (LUT) return 0u;
+    const uint32_t os = rit32((uint32_t)rb * 32 + lane, 2 * uk, p.rb.scales);
+    return CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_SCALES], 209) ? ldg_u16(p.scales + os) : 0u;
   }
   static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
 #pragma unroll
@@ -339,9 +353,14 @@ struct UnitBitmap {
   static CQL_DEV void on_row(const DecodeParams&, uint8_t*, int, int) {}
   static constexpr int kSlabs = 1;                        // the unit's bitmap slab
   static CQL_DEV uint32_t issue(const DecodeParams& p, int rb, int uk, int lane, uint8_t* slot) {
-    cp_async16(slot, p.meta + slab_off(rb, uk, p.rb.meta) + lane * 16);
+    const uint64_t om = slab_off(rb, uk, p.rb.meta) + lane * 16;
+    if (CQL_IN(p.err, om + 15, p.plane_len[CQL_PLANE_META], 210)) cp_async16(slot, p.meta + om);
     const uint64_t row = (uint64_t)rb * 32 + lane;
-    return ldg_u16(p.voff + rit(row, 2 * uk, p.rb.voff)) | (ldg_u16(p.scales + rit(row, 2 * uk, p.rb.scales)) << 16);
+    const uint64_t oo = rit(row, 2 * uk, p.rb.voff), os = rit(row, 2 * uk, p.rb.scales);
+    if (!CQL_IN(p.err, oo + 1, p.plane_len[CQL_PLANE_VOFF], 211) ||
+        !CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_SCALES], 212))
+      return 0u;
+    return ldg_u16(p.voff + oo) | (ldg_u16(p.scales + os) << 16);
   }
   static CQL_DEV void gather(const uint8_t* slot, uint32_t sc, Frag& f) {
     const uint4 m = lds128(slot);
@@ -360,7 +379,9 @@ struct UnitBitmap {
 #pragma unroll
     for (int s = 0; s < kWinWords / 4; ++s) {
       const uint32_t sl = min((bo >> 4) + s, nslab - 1);
-      const uint4 a = ldg_stream(p.values + slab_off(rb, sl, p.rb.values) + lane * 16);
+      const uint64_t ov = slab_off(rb, sl, p.rb.values) + lane * 16;
+      const uint4 a = CQL_IN(p.err, ov + 15, p.plane_len[CQL_PLANE_VALUES], 213) ? ldg_stream(p.values + ov)
+                                                                                 : make_uint4(0u, 0u, 0u, 0u);
       win[(4 * s + 0) * 32 + lane] = a.x; win[(4 * s + 1) * 32 + lane] = a.y;
       win[(4 * s + 2) * 32 + lane] = a.z; win[(4 * s + 3) * 32 + lane] = a.w;
     }
@@ -537,10 +558,14 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
   uint8_t* lsm = esm + (size_t)B * p.r_pad * 4;
   uint16_t* ssm = reinterpret_cast<uint16_t*>(lsm + (size_t)nch * kEpiThreads * 16);   // s_L[g][0 .. r)
   if (lowrank) {
-    for (int m = 0; m < nch; ++m)
-      cp_async16(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16, p.l_values + slab_off(rb, m, p.rb.l_values) + lane * 16);
+    for (int m = 0; m < nch; ++m) {
+      const uint64_t ol = slab_off(rb, m, p.rb.l_values) + lane * 16;
+      if (CQL_IN(p.err, ol + 15, p.plane_len[CQL_PLANE_L_VALUES], 214))
+        cp_async16(lsm + ((size_t)m * kEpiThreads + threadIdx.x) * 16, p.l_values + ol);
+    }
     for (int i = threadIdx.x; i < r / 2; i += kEpiThreads)   // r is a multiple of 16
-      cp_async4(ssm + 2 * i, p.l_scales + (uint64_t)g * r + 2 * i);
+      if (CQL_IN(p.err, 2 * ((uint64_t)g * r + 2 * i) + 3, p.plane_len[CQL_PLANE_L_SCALES], 215))
+        cp_async4(ssm + 2 * i, p.l_scales + (uint64_t)g * r + 2 * i);
   }
   cp_async_commit();
   pdl_wait();                                       // main term (and pre-kernel) complete
@@ -548,7 +573,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
 #pragma unroll
   for (int b = 0; b < B; ++b) {
     acc[b] = 0.0f;
-    if (b < p.batch) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
+    if (b < p.batch && CQL_IN(p.err, (uint64_t)b * N + row, p.y_elems, 216)) acc[b] = ld_cg_f32(p.y_acc + (uint64_t)b * N + row);
   }
   if (lowrank) {
     cp_async_wait<0>();
@@ -563,7 +588,10 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
       for (int j = threadIdx.x; j < r; j += kEpiThreads) {
         float v[B];
 #pragma unroll
-        for (int b = 0; b < B; ++b) v[b] = b < p.batch ? ld_cg_f32(tfin + (uint64_t)b * p.r_pad + j) : 0.0f;
+        for (int b = 0; b < B; ++b)
+          v[b] = b < p.batch && CQL_IN(p.err, (uint64_t)(tfin - p.t_final) + (uint64_t)b * p.r_pad + j, p.t_final_elems, 217)
+                     ? ld_cg_f32(tfin + (uint64_t)b * p.r_pad + j)
+                     : 0.0f;
         const float sl = f16_bits_to_f32(ssm[j]);
 #pragma unroll
         for (int b = 0; b < B; ++b) us[b * r + j] = sl * v[b];
@@ -575,6 +603,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
       const float* tp = p.t_part + (uint64_t)b * p.r_pad + j;
       const uint64_t st = (uint64_t)B * p.r_pad;
       int k = 0;
+      if (!CQL_IN(p.err, (uint64_t)(tp - p.t_part) + (uint64_t)(kq - 1) * st, p.t_part_elems, 218)) k = kq;   // skip
       for (; k + 4 <= kq; k += 4) {
         t0 += ld_cg_f32(tp + (k + 0) * st);
         t1 += ld_cg_f32(tp + (k + 1) * st);
@@ -588,7 +617,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
   __syncthreads();
 #pragma unroll
   for (int b = 0; b < B; ++b)
-    if (b < p.batch) p.y_acc[(uint64_t)b * N + row] = 0.0f;
+    if (b < p.batch && CQL_IN(p.err, (uint64_t)b * N + row, p.y_elems, 219)) p.y_acc[(uint64_t)b * N + row] = 0.0f;
   if (lowrank && B >= 8) {
     cp_async_wait<0>();
     // 8 and more batch rows: every code is converted once per 8 batch rows,
@@ -651,7 +680,7 @@ __global__ void __maxnreg__(64) k_epilogue(DecodeParams p, int kq) {
   }
 #pragma unroll
   for (int b = 0; b < B; ++b)
-    if (b < p.batch) store_out(p.y, p.ydt, (uint64_t)b * N + row, acc[b]);
+    if (b < p.batch && CQL_IN(p.err, (uint64_t)b * N + row, p.y_elems, 220)) store_out(p.y, p.ydt, (uint64_t)b * N + row, acc[b]);
 }
 
 // ---------------------------------------------------------------------------
@@ -682,10 +711,12 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
     uint4 q4[4];
     float sc = 0.0f;
     if (u < u1) {                                     // R codes first: they do not depend on x
-      const uint8_t* base = p.r_values + slab_off(rbR, 4 * u, p.rb.r_values) + lane * 16;
+      const uint64_t ob = slab_off(rbR, 4 * u, p.rb.r_values) + lane * 16;
+      const uint64_t os = rit(j, 2 * u, p.rb.r_scales);
+      const bool okv = CQL_IN(p.err, ob + 3 * 512 + 15, p.plane_len[CQL_PLANE_R_VALUES], 221);
 #pragma unroll
-      for (int s = 0; s < 4; ++s) q4[s] = ldg_stream(base + 512 * s);
-      sc = f16_bits_to_f32(ldg_u16(p.r_scales + rit(j, 2 * u, p.rb.r_scales)));
+      for (int s = 0; s < 4; ++s) q4[s] = okv ? ldg_stream(p.r_values + ob + 512 * s) : make_uint4(0u, 0u, 0u, 0u);
+      sc = CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_R_SCALES], 222) ? f16_bits_to_f32(ldg_u16(p.r_scales + os)) : 0.0f;
     }
     stage_x<B>(p, s1, u0 * kGroup, (u1 - u0) * kGroup);
     __syncthreads();
@@ -719,11 +750,13 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
       float t = 0.0f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) t += s1[(w * B + b) * 32 + l];
-      p.t_part[((uint64_t)kq * B + b) * p.r_pad + 32 * rbR + l] = t;
+      if (CQL_IN(p.err, ((uint64_t)kq * B + b) * p.r_pad + 32 * rbR + l, p.t_part_elems, 223))
+        p.t_part[((uint64_t)kq * B + b) * p.r_pad + 32 * rbR + l] = t;
     }
   } else {
     const int row = (blockIdx.x - n_s1) * blockDim.x + threadIdx.x;
     if (row >= p.d.n_out) return;
+    if (!CQL_IN(p.err, 4ull * row + 7, p.plane_len[CQL_PLANE_CSR_ROWPTR], 224)) return;
     int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
     e0 = max(0, min(e0, (int)p.nnz));
     e1 = max(e0, min(e1, (int)p.nnz));
@@ -748,7 +781,8 @@ __global__ void __launch_bounds__(256, 1) k_pre(DecodeParams p, int n_s1) {
     }
 #pragma unroll
     for (int b = 0; b < B; ++b)
-      if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
+      if (b < p.batch && CQL_IN(p.err, (uint64_t)b * p.d.n_out + row, p.y_elems, 225))
+        atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
   }
 }
 

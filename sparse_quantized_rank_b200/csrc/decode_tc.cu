@@ -200,8 +200,10 @@ CQL_DEV SideFirst tc_side_prefetch(const DecodeParams& p, int iw, int lane) {
   const int it = iw * gridDim.x + blockIdx.x;
   if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK) && it < (p.r_pad / 32) * (K / 32)) {
     const int s32 = it % (K / 32), rbr = it / (K / 32);
-    f.q4 = ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
-    f.sc = ldg_u16(p.r_scales + rit32((uint32_t)(32 * rbr + lane), 2u * (s32 >> 2), p.rb.r_scales));
+    const uint32_t ov = slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16;
+    const uint32_t os = rit32((uint32_t)(32 * rbr + lane), 2u * (s32 >> 2), p.rb.r_scales);
+    if (CQL_IN(p.err, ov + 15, p.plane_len[CQL_PLANE_R_VALUES], 101)) f.q4 = ldg_stream(p.r_values + ov);
+    if (CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_R_SCALES], 102)) f.sc = ldg_u16(p.r_scales + os);
   }
   return f;
 }
@@ -218,12 +220,14 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
   {
     float* t_old = p.t_final + (size_t)(par ^ 1u) * B * p.r_pad;
     const int tot = B * p.r_pad, per = (tot + gridDim.x - 1) / gridDim.x;
-    for (int i = blockIdx.x * per + iw * 32 + lane; i < min(tot, (int)(blockIdx.x + 1) * per); i += NW * 32) t_old[i] = 0.0f;
+    for (int i = blockIdx.x * per + iw * 32 + lane; i < min(tot, (int)(blockIdx.x + 1) * per); i += NW * 32)
+      if (CQL_IN(p.err, (uint64_t)(t_old - p.t_final) + i, p.t_final_elems, 103)) t_old[i] = 0.0f;
     if (blockIdx.x == 0 && iw == 0 && lane == 0) p.t_counter[1] = par;
   }
   if (p.csr_rowptr != nullptr && !(p.flags & CQL_FLAG_NO_CSR)) {
     const int r0 = (int)((uint64_t)N * blockIdx.x / gridDim.x), r1 = (int)((uint64_t)N * (blockIdx.x + 1) / gridDim.x);
     for (int row = r0 + iw * 32 + lane; row < r1; row += NW * 32) {
+      if (!CQL_IN(p.err, 4ull * row + 7, p.plane_len[CQL_PLANE_CSR_ROWPTR], 104)) continue;
       int e0 = p.csr_rowptr[row], e1 = p.csr_rowptr[row + 1];
       e0 = max(0, min(e0, (int)p.nnz));
       e1 = max(e0, min(e1, (int)p.nnz));
@@ -237,11 +241,13 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
         const float v = f16_bits_to_f32(p.csr_val[e]);
 #pragma unroll
         for (int b = 0; b < B; ++b)
-          if (b < p.batch) acc[b] = fmaf(v, to_f32_act(p.x, p.xdt, (uint64_t)b * K + col), acc[b]);
+          if (b < p.batch && CQL_IN(p.err, (uint64_t)b * K + col, p.x_elems, 105))
+            acc[b] = fmaf(v, to_f32_act(p.x, p.xdt, (uint64_t)b * K + col), acc[b]);
       }
 #pragma unroll
       for (int b = 0; b < B; ++b)
-        if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * N + row, acc[b]);
+        if (b < p.batch && CQL_IN(p.err, (uint64_t)b * N + row, p.y_elems, 106))
+          atomicAdd(p.y_acc + (uint64_t)b * N + row, acc[b]);
     }
   }
   if (p.d.rank > 0 && !(p.flags & CQL_FLAG_NO_LOWRANK)) {
@@ -253,13 +259,19 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
       const int s32 = it % (K / 32), rbr = it / (K / 32);
       const int j = 32 * rbr + lane, u = s32 >> 2;
       const bool pre = it == iw * (int)gridDim.x + (int)blockIdx.x;   // the prefetched first item
-      const uint4 q4 = pre ? first.q4 : ldg_stream(p.r_values + slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16);
-      const float sc = f16_bits_to_f32(pre ? first.sc : ldg_u16(p.r_scales + rit32((uint32_t)j, 2u * u, p.rb.r_scales)));
+      const uint32_t ov = slab_off32((uint32_t)rbr, (uint32_t)s32, p.rb.r_values) + lane * 16;
+      const uint32_t os = rit32((uint32_t)j, 2u * u, p.rb.r_scales);
+      const uint4 q4 = pre ? first.q4
+                           : (CQL_IN(p.err, ov + 15, p.plane_len[CQL_PLANE_R_VALUES], 107) ? ldg_stream(p.r_values + ov)
+                                                                                           : make_uint4(0u, 0u, 0u, 0u));
+      const float sc = f16_bits_to_f32(
+          pre ? first.sc
+              : (CQL_IN(p.err, os + 1, p.plane_len[CQL_PLANE_R_SCALES], 108) ? ldg_u16(p.r_scales + os) : 0u));
       float xv[B];                                  // x[b][32 s32 + lane]
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         xv[b] = 0.0f;
-        if (b < p.batch) {
+        if (b < p.batch && CQL_IN(p.err, (uint64_t)b * K + 32 * s32 + lane, p.x_elems, 109)) {
           const uint32_t xh = static_cast<const uint16_t*>(p.x)[(uint64_t)b * K + 32 * s32 + lane];
           xv[b] = p.xdt == CQL_DT_BF16 ? bf16_bits_to_f32(xh) : f16_bits_to_f32(xh);
         }
@@ -277,7 +289,9 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
       if (j < p.d.rank) {
 #pragma unroll
         for (int b = 0; b < B; ++b)
-          if (b < p.batch) atomicAdd(t_acc + (uint64_t)b * p.r_pad + j, sc * a[b]);
+          if (b < p.batch &&
+              CQL_IN(p.err, (uint64_t)(t_acc - p.t_final) + (uint64_t)b * p.r_pad + j, p.t_final_elems, 110))
+            atomicAdd(t_acc + (uint64_t)b * p.r_pad + j, sc * a[b]);
       }
     }
   }
@@ -417,12 +431,24 @@ __global__ void __maxnreg__(88)
     ld.init(geo, t0 + w);
     auto fetch = [&](int slot_i) {
       const uint32_t rb = 4u * ld.rt + qq;
-      const uint8_t* vsrc = p.values + rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
       uint8_t* slot = ring + slot_i * TC_SLOT_BYTES;
+#ifdef CQL_CHECKED
+      const uint32_t ov = rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
+      const uint32_t om = rb * mstride + (uint32_t)ld.g * 512u + lane * 16;
+      const uint32_t os = rb * sstride + (uint32_t)(ld.g >> 3) * 512u + lane * 16;
+      if (CQL_IN(p.err, ov + 512 + 15, p.plane_len[CQL_PLANE_VALUES], 111)) {
+        cp_async16(slot, p.values + ov);
+        cp_async16(slot + 512, p.values + ov + 512);
+      }
+      if (CQL_IN(p.err, om + 15, p.plane_len[CQL_PLANE_META], 112)) cp_async16(slot + 1024, p.meta + om);
+      if (CQL_IN(p.err, os + 15, p.plane_len[CQL_PLANE_SCALES], 113)) cp_async16(slot + 1536, p.scales + os);
+#else
+      const uint8_t* vsrc = p.values + rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
       cp_async16(slot, vsrc);
       cp_async16(slot + 512, vsrc + 512);
       cp_async16(slot + 1024, p.meta + rb * mstride + (uint32_t)ld.g * 512u + lane * 16);
       cp_async16(slot + 1536, p.scales + rb * sstride + (uint32_t)(ld.g >> 3) * 512u + lane * 16);
+#endif
       if (lane == 0) {
         S.slot_rt[cw][slot_i] = ld.rt;
         S.slot_g[cw][slot_i] = ld.g;
@@ -474,7 +500,8 @@ __global__ void __maxnreg__(88)
           }
 #pragma unroll
           for (int b = 0; b < B; ++b) {
-            if (b < p.batch) atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
+            if (b < p.batch && CQL_IN(p.err, (uint64_t)b * p.d.n_out + row, p.y_elems, 114))
+              atomicAdd(p.y_acc + (uint64_t)b * p.d.n_out + row, acc[b]);
             acc[b] = 0.0f;
           }
         }

@@ -88,6 +88,10 @@ struct DecodeParams {
   const uint8_t* l_values;
   const uint16_t* l_scales;
   uint64_t nnz;
+  uint64_t plane_len[CQL_NPLANES];   // bytes of every plane (the checked build's bounds)
+  uint64_t x_elems, y_elems;         // batch * K, batch * N
+  uint64_t t_final_elems;            // floats in t_final
+  uint64_t t_part_elems;             // floats in t_part
   const void* x;
   int xdt;
   void* y;

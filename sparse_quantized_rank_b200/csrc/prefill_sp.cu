@@ -88,9 +88,10 @@ struct SpParams {
   void* out;                  // y [m][N]
   int out_dt;
   uint32_t* err;
+  uint64_t len_values, len_meta, len_scales;   // plane bytes (the checked build's bounds)
 };
 
-// Instruction descriptors (M = 128, N = 192, D f32, A = B = bf16 or f16,
+// Instruction descriptors (M = 128, N = 208, D f32, A = B = bf16 or f16,
 // both K-major): sparse for the quantised term, dense for the adapter blocks.
 CQL_HD uint32_t sp_idesc(bool f16, bool sparse) {
   const uint32_t fmt = f16 ? 0u : 1u;
@@ -228,11 +229,15 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       if (mg == 0 || f_tile >= my_tiles) return;
       const int item = blockIdx.x + f_tile * gridDim.x;
       const uint32_t rbk = 4u * (uint32_t)(item / p.tok_tiles) + qq;
-      const uint8_t* vsrc = p.values + rbk * vstride + (uint32_t)f_g * 1024u + lane * 16;
+      const uint32_t ov = rbk * vstride + (uint32_t)f_g * 1024u + lane * 16;
+      const uint32_t om = rbk * mstride + (uint32_t)f_g * 512u + lane * 16;
+      const uint8_t* vsrc = p.values + ov;
       uint8_t* sl = ring + slot * SP_RAW;
-      cp_async16(sl, vsrc);
-      cp_async16(sl + 512, vsrc + 512);
-      cp_async16(sl + 1024, p.meta + rbk * mstride + (uint32_t)f_g * 512u + lane * 16);
+      if (CQL_IN(p.err, ov + 512 + 15, p.len_values, 301)) {
+        cp_async16(sl, vsrc);
+        cp_async16(sl + 512, vsrc + 512);
+      }
+      if (CQL_IN(p.err, om + 15, p.len_meta, 302)) cp_async16(sl + 1024, p.meta + om);
       if (++f_g == mg) {
         f_g = 0;
         ++f_tile;
@@ -309,7 +314,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < SP_EPI_COLS; ++i) acc[i] = 0.0f;
       auto scale_of = [&](int g) {
-        return g < mg ? f16_bits_to_f32(ldg_u16(p.scales + rit32((uint32_t)row, 2u * g, p.rb.scales))) : 1.0f;
+        const uint32_t os = rit32((uint32_t)row, 2u * g, p.rb.scales);
+        return g < mg ? (CQL_IN(p.err, os + 1, p.len_scales, 303) ? f16_bits_to_f32(ldg_u16(p.scales + os)) : 0.0f)
+                      : 1.0f;
       };
       float s_next = ngroups > 0 ? scale_of(0) : 1.0f;
       for (int g = 0; g < ngroups; ++g, ++gc) {
@@ -355,7 +362,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       const int t0 = tt * SP_BN + h * SP_EPI_COLS;
 #pragma unroll
       for (int i = 0; i < SP_EPI_COLS; ++i)
-        if (t0 + i < p.m) store_out(p.out, p.out_dt, (uint64_t)(t0 + i) * p.rows + row, acc[i]);
+        if (t0 + i < p.m && CQL_IN(p.err, (uint64_t)(t0 + i) * p.rows + row, (uint64_t)p.m * p.rows, 304))
+          store_out(p.out, p.out_dt, (uint64_t)(t0 + i) * p.rows + row, acc[i]);
     }
     if (!ok && lane == 0) set_error(p.err, CQL_ERR_TIMEOUT, 33);
   }
@@ -413,6 +421,9 @@ static cudaError_t launch_sg(const DecodeParams& p, const uint16_t* lbuf, int r3
   s.row_tiles = N / SP_BM;
   s.tok_tiles = (m + SP_BN - 1) / SP_BN;
   s.out = p.y;
+  s.len_values = p.plane_len[CQL_PLANE_VALUES];
+  s.len_meta = p.plane_len[CQL_PLANE_META];
+  s.len_scales = p.plane_len[CQL_PLANE_SCALES];
   s.out_dt = p.ydt;
   s.err = p.err;
   const int items = s.row_tiles * s.tok_tiles;

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(256) k_sal_scale_w(const void* W, int wdt, uin
 // blockIdx.y + gridDim.y, ...  The list is staged before the dependency wait
 // (the packed buffer is not written by the preceding kernel); x only after.
 __global__ void __launch_bounds__(256) k_salient_x(const uint16_t* list, int m, int K, int batch, int xdt,
-                                                   int log2, const uint16_t* x, uint16_t* xs) {
+                                                   int log2, const uint16_t* x, uint16_t* xs, uint32_t* err) {
   extern __shared__ uint16_t sl[];
   pdl_launch_dependents();
   for (int i = threadIdx.x; i < m; i += blockDim.x) sl[i] = list[i];
@@ -127,12 +127,14 @@ __global__ void __launch_bounds__(256) k_salient_x(const uint16_t* list, int m, 
   const float inv = ldexpf(1.0f, -log2);
   for (int b = blockIdx.y; b < batch; b += gridDim.y) {
     const uint64_t off = (uint64_t)b * K + 8u * (uint32_t)v;
+    if (!CQL_IN(err, off + 7, (uint64_t)batch * K, 401)) continue;
     uint4 q = *reinterpret_cast<const uint4*>(x + off);
     if (any) {
       uint16_t h[8];
       memcpy(h, &q, 16);
       for (int j = lo; j < m && (int)sl[j] < 8 * v + 8; ++j) {
         const int e = sl[j] - 8 * v;
+        if (!CQL_IN(err, (uint64_t)e, 8, 402)) continue;
         if (xdt == CQL_DT_BF16) {
           h[e] = __bfloat16_as_ushort(__float2bfloat16_rn(bf16_bits_to_f32(h[e]) * inv));
         } else {
@@ -179,7 +181,7 @@ cudaError_t launch_salient_x(const DecodeParams& p, const uint16_t* list, void* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_salient_x, list, m, K, (int)p.batch, (int)p.xdt, (int)p.d.salient_log2,
-                            static_cast<const uint16_t*>(p.x), static_cast<uint16_t*>(xs));
+                            static_cast<const uint16_t*>(p.x), static_cast<uint16_t*>(xs), p.err);
 }
 
 }  // namespace cql

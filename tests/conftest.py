@@ -19,3 +19,19 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the session's per-config parity errors and oracle times as JSON
+    lines when CQL_METRICS_JSONL names a file."""
+    path = os.environ.get("CQL_METRICS_JSONL")
+    if not path:
+        return
+    try:
+        from tests.gpu_util import METRICS
+    except Exception:
+        return
+    import json
+    with open(path, "w") as f:
+        for m in METRICS:
+            f.write(json.dumps(m) + "\n")

@@ -1,6 +1,8 @@
 """Helpers for the GPU parity tests: move seeded inputs to the device, run the
 library through its C ABI, and compare with the oracle."""
 import math
+import os
+import time
 
 import numpy as np
 
@@ -9,6 +11,11 @@ import sparse_quantized_rank_b200 as C
 from workloads import make_layer_inputs
 
 DT_NAME = {C.CQL_DT_F32: "f32", C.CQL_DT_F16: "f16", C.CQL_DT_BF16: "bf16"}
+
+# Per-config metrics of this session (written as JSON lines by conftest when
+# CQL_METRICS_JSONL names a file): every parity comparison's max relative
+# error, and the oracle's time for every reference forward.
+METRICS = []
 
 
 def c_desc(od: O.OracleDesc, flags: int = 0):
@@ -58,7 +65,12 @@ class Case:
         return y
 
     def reference(self, batch, flags=0):
-        return O.forward(self.parts, self.inp["x"][:batch].astype(np.float64), flags=flags)
+        t0 = time.perf_counter()
+        y = O.forward(self.parts, self.inp["x"][:batch].astype(np.float64), flags=flags)
+        METRICS.append({"kind": "oracle_time", "workload": self.wl.name, "n": self.wl.n, "k": self.wl.k,
+                        "batch": int(batch), "flags": int(flags), "oracle_ms": (time.perf_counter() - t0) * 1e3,
+                        "threads": os.cpu_count()})
+        return y
 
 
 def half_ulp(ref: np.ndarray, dt: str) -> np.ndarray:
@@ -91,4 +103,7 @@ def check_close(y, ref, dt: str, tol: float = 2e-3, what: str = ""):
         raise AssertionError(f"{what}: {int(bad.sum())} of {err.size} outside tolerance; worst at {i}: "
                              f"y={yv[i]!r} ref={ref[i]!r} err={err[i]:.3e} bound={bound[i]:.3e} "
                              f"rel_err={O.rel_err(yv, ref):.3e}")
-    return O.rel_err(yv, ref)
+    r = O.rel_err(yv, ref)
+    METRICS.append({"kind": "parity", "what": what, "out_dtype": dt, "max_rel_err": r, "tol": tol,
+                    "elements": int(err.size)})
+    return r

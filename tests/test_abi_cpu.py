@@ -38,6 +38,23 @@ def test_exports_every_declared_symbol(lib):
     assert C.cql_status_string(C.CQL_ERR_SIZE).startswith("CQL_ERR_SIZE")
 
 
+def test_checked_build_exports_every_declared_symbol():
+    """The range-checked variant (-DCQL_CHECKED) builds and exports the same
+    C ABI; selecting it routes the binding's calls to it."""
+    path = B.build(checked=True)
+    assert path.endswith("libcql_checked.so")
+    L = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(L, n), n
+    C.use_library(True)
+    try:
+        assert C.cql_status_string(C.CQL_ERR_RANGE).startswith("CQL_ERR_RANGE")
+        assert C.lib()._name == path
+    finally:
+        C.use_library(False)
+    assert C.lib()._name.endswith("libcql.so")
+
+
 def test_desc_struct_size():
     assert ctypes.sizeof(C.cql_desc) == 64
     assert ctypes.sizeof(C.cql_layout) == 16 + 2 * 8 * 13
