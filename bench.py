@@ -475,9 +475,11 @@ def run_cql(args):
             "peak_source": f"{tf_src} dense bf16 (MEASURED_PEAKS.json bf16_tflops)",
             "kernel": "k_pf_sgemm (tcgen05.mma.sp, codes converted on chip) after the adapter passes; achieved = "
                       "dense-equivalent 2MNK per call / whole-call time",
-            "sparse_frac": algo / per_step / 1e12 / (2 * tf_peak),
-            "sparse_note": "algorithmic flops (MNK on the kept half plus the adapter product) against twice the "
-                           "dense peak (the sparse tensor-core rate)"}
+            "sparse_frac": dense / per_step / 1e12 / (2 * tf_peak),
+            "sparse_note": "dense-equivalent flops against twice the dense peak (the 2:4 sparse tensor cores "
+                           "execute a logical K at twice the dense rate); equally, algorithmic flops (the kept "
+                           "half plus the adapter product) against the dense peak",
+            "algorithmic_tflops": algo / per_step / 1e12}
         line["kernels_per_step"] = "k_pf_dequant_l, k_pf_dequant_r, k_pf_gemm (T), k_pf_tsplit, k_pf_sgemm"
     del b
     torch.cuda.empty_cache()

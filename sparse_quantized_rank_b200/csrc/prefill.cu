@@ -309,66 +309,76 @@ __global__ void k_pf_dequant_w(DecodeParams p, uint16_t* qbf, int ldq, float* sc
   scales[(uint64_t)n * G + g] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(p.scales + rit(n, 2 * g, p.rb.scales)));
 }
 
-// Adapter columns of the main operand: [Lhi | Lhi | Llo | 0] at columns
-// col0 .. col0 + r3 of row n, with L^ = q_L s_L exact in fp32 and
-// Lhi + Llo = L^ (col0 = K after the dense codes; 0 in the separate adapter
-// buffer of the sparse GEMM).
-// A thread per (row, 8 columns): one 16-byte store.
-__global__ void k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int col0, int r3, int f16) {
-  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int r = p.d.rank, chunks = r3 / 8;
-  if (id >= (uint64_t)p.d.n_out * chunks) return;
-  const int n = (int)(id / chunks), c0 = (int)(id % chunks) * 8;
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = c0 + i;
-    uint32_t v = 0;
-    if (c < 3 * r) {
-      const int j = c % r, part = c / r;               // 0: hi, 1: hi, 2: lo
-      const uint32_t byte = p.l_values[rit(n, j / 2, p.rb.l_values)];
-      const int q = (int)((byte >> (4 * (j & 1))) & 15u) - 8;
-      const float sl = f16_bits_to_f32(p.l_scales[(uint64_t)(n / kGroup) * r + j]);
-      const float l = (float)q * sl;                     // exact (<= 14 significant bits)
-      const uint16_t hi = to16(l, f16);
-      v = part < 2 ? hi : to16(l - from16(hi, f16), f16);
-    }
-    w[i >> 1] |= v << (16 * (i & 1));
+// L (N x r) as exact bf16 (f16) hi / hi / lo columns [N][r3] (zero padding
+// up to r3): a warp per row, lane = column pairs (2j, 2j + 1), each part
+// written as one coalesced run of 4-byte pairs.
+__global__ void __launch_bounds__(256) k_pf_dequant_l(DecodeParams p, uint16_t* qbf, int ldq, int col0, int r3,
+                                                      int f16) {
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (n >= p.d.n_out) return;
+  const int r = p.d.rank;
+  uint16_t* out = qbf + (uint64_t)n * ldq + col0;
+  const uint16_t* sl = p.l_scales + (uint64_t)(n / kGroup) * r;
+  for (int j = 2 * lane; j < r; j += 64) {
+    const uint32_t byte = p.l_values[rit(n, j / 2, p.rb.l_values)];
+    const float l0 = (float)((int)(byte & 15u) - 8) * f16_bits_to_f32(sl[j]);       // exact
+    const float l1 = (float)((int)(byte >> 4) - 8) * f16_bits_to_f32(sl[j + 1]);
+    const uint32_t h0 = to16(l0, f16), h1 = to16(l1, f16);
+    const uint32_t hi = h0 | (h1 << 16);
+    const uint32_t lo = (uint32_t)to16(l0 - from16((uint16_t)h0, f16), f16) |
+                        ((uint32_t)to16(l1 - from16((uint16_t)h1, f16), f16) << 16);
+    *reinterpret_cast<uint32_t*>(out + j) = hi;
+    *reinterpret_cast<uint32_t*>(out + r + j) = hi;
+    *reinterpret_cast<uint32_t*>(out + 2 * r + j) = lo;
   }
-  *reinterpret_cast<uint4*>(qbf + (uint64_t)n * ldq + col0 + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int c = 3 * r + 2 * lane; c < r3; c += 64) *reinterpret_cast<uint32_t*>(out + c) = 0u;
 }
 
-// R rows (padded to 128) as bf16 codes and fp32 scales.
-__global__ void k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, int rows, int f16) {
+// R rows (padded to 128) as bf16 (f16) codes and fp32 scales: a thread per
+// 16 codes (8 bytes of a row, one half of a 16-byte piece of the plane).
+__global__ void __launch_bounds__(256) k_pf_dequant_r(DecodeParams p, uint16_t* rbf, float* rscales, int rows,
+                                                      int f16) {
   const int K = p.d.k_in, G = p.upr;
   const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= (uint64_t)rows * K) return;
-  const int j = (int)(id / K), k = (int)(id % K);
-  uint16_t v = 0;
+  if (id >= (uint64_t)rows * (K / 16)) return;
+  const int j = (int)(id / (K / 16)), k0 = (int)(id % (K / 16)) * 16;
+  uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   if (j < p.d.rank) {
-    const uint32_t byte = p.r_values[rit(j, k / 2, p.rb.r_values)];
-    v = int_to16((int)((byte >> (4 * (k & 1))) & 15u) - 8, f16);
+    const uint2 b8 = *reinterpret_cast<const uint2*>(p.r_values + rit(j, k0 / 2, p.rb.r_values));
+    const uint32_t bw[2] = {b8.x, b8.y};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t byte = (bw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+      w[i] = (uint32_t)int_to16((int)(byte & 15u) - 8, f16) | ((uint32_t)int_to16((int)(byte >> 4) - 8, f16) << 16);
+    }
   }
-  rbf[id] = v;
-  if (k % kGroup == 0)
-    rscales[(uint64_t)j * G + k / kGroup] =
-        j < p.d.rank ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(p.r_scales + rit(j, 2 * (k / kGroup), p.rb.r_scales)))
+  uint4* dst = reinterpret_cast<uint4*>(rbf + (uint64_t)j * K + k0);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  if (k0 % kGroup == 0)
+    rscales[(uint64_t)j * G + k0 / kGroup] =
+        j < p.d.rank ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(p.r_scales + rit(j, 2 * (k0 / kGroup), p.rb.r_scales)))
                      : 0.0f;
 }
 
-// T [m][r_pad] fp32 -> [Thi | Tlo | Thi | 0] as bf16 (or fp16) [m][r3].
-__global__ void k_pf_tsplit(const float* t, int ldt, uint16_t* t3, int r3, int r, int m, int f16) {
-  const uint64_t id = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= (uint64_t)m * r3) return;
-  const int row = (int)(id / r3), c = (int)(id % r3);
-  uint16_t v = 0;
-  if (c < 3 * r) {
-    const int j = c % r, part = c / r;                       // 0: hi, 1: lo, 2: hi
-    const float x = t[(uint64_t)row * ldt + j];
-    const uint16_t hi = to16(x, f16);
-    v = part == 1 ? to16(x - from16(hi, f16), f16) : hi;
+// T [m][r_pad] fp32 -> [Thi | Tlo | Thi | 0] as bf16 (or fp16) [m][r3]: a
+// warp per token row, lane = column pairs.
+__global__ void __launch_bounds__(256) k_pf_tsplit(const float* t, int ldt, uint16_t* t3, int r3, int r, int m,
+                                                   int f16) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= m) return;
+  uint16_t* out = t3 + (uint64_t)row * r3;
+  for (int j = 2 * lane; j < r; j += 64) {
+    const float2 x = *reinterpret_cast<const float2*>(t + (uint64_t)row * ldt + j);
+    const uint32_t h0 = to16(x.x, f16), h1 = to16(x.y, f16);
+    const uint32_t hi = h0 | (h1 << 16);
+    const uint32_t lo = (uint32_t)to16(x.x - from16((uint16_t)h0, f16), f16) |
+                        ((uint32_t)to16(x.y - from16((uint16_t)h1, f16), f16) << 16);
+    *reinterpret_cast<uint32_t*>(out + j) = hi;
+    *reinterpret_cast<uint32_t*>(out + r + j) = lo;
+    *reinterpret_cast<uint32_t*>(out + 2 * r + j) = hi;
   }
-  t3[id] = v;
+  for (int c = 3 * r + 2 * lane; c < r3; c += 64) *reinterpret_cast<uint32_t*>(out + c) = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -445,9 +455,8 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
     if (!main_on) cudaMemsetAsync(wsc, 0, (uint64_t)N * G * 4, st);     // main term off: zero scales
   }
   if (lowrank) {
-    const uint64_t nl = (uint64_t)N * (L.r3 / 8);
-    k_pf_dequant_l<<<(unsigned)((nl + 255) / 256), 256, 0, st>>>(p, qbf, L.ldq, L.sparse ? 0 : K, L.r3, f16);
-    const uint64_t nr = (uint64_t)L.rrows * K;
+    k_pf_dequant_l<<<(unsigned)((N + 7) / 8), 256, 0, st>>>(p, qbf, L.ldq, L.sparse ? 0 : K, L.r3, f16);
+    const uint64_t nr = (uint64_t)L.rrows * (K / 16);
     k_pf_dequant_r<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(p, rbf, rsc, L.rrows, f16);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -468,8 +477,7 @@ cudaError_t launch_prefill(const DecodeParams& p, uint8_t* pws, cudaStream_t st)
     t.err = p.err;
     const int items = tiles * t.k_splits;
     k_pf_gemm<<<min(items, sms), PF_THREADS, smem, st>>>(mR, mB, mB, t);
-    const uint64_t nt = (uint64_t)m * L.r3;
-    k_pf_tsplit<<<(unsigned)((nt + 255) / 256), 256, 0, st>>>(tacc, L.r_pad, t3, L.r3, r, m, f16);
+    k_pf_tsplit<<<(unsigned)((m + 7) / 8), 256, 0, st>>>(tacc, L.r_pad, t3, L.r3, r, m, f16);
     if (!make_map(&mT, t3, (uint64_t)m, (uint64_t)L.r3, (uint64_t)L.r3, PF_BN)) return cudaErrorInvalidValue;
   } else {
     mT = mB;
