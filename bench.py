@@ -123,7 +123,7 @@ def kernels_per_step(wl, batch):
     pro = 1 if wl.salient_channels else 0
     if batch > 16:                       # prefill: adapter passes (4 kernels) and the main GEMM
         return pro + 1 + (4 if wl.rank else 0) + (0 if (wl.mask == "2:4" and wl.codec == "int4") else 1)
-    if wl.mask == "2:4" and wl.codec == "int4":
+    if wl.mask == "2:4" and wl.codec in ("int4", "int3"):
         return 2 + pro
     return 2 + pro + (1 if (wl.rank or wl.outlier_frac) else 0)
 
@@ -514,8 +514,8 @@ def extra_lines(torch, C, dev, stream, barrier):
     peak, _ = measured_peaks()
     for name, batch in (("mlp_up", 1), ("tiny", 1), ("mlp_up", 4), ("mlp_up", 16), ("lut_dense_sparse", 1),
                         ("lut_dense_sparse", 8), ("down_unstructured", 1), ("down_unstructured", 16),
-                        ("mlp_up_slimo", 1), ("mlp_up_slimo", 16)):
-        wl = workload(name)
+                        ("mlp_up_slimo", 1), ("mlp_up_slimo", 16), ("mlp_up_int3", 1), ("mlp_up_int3", 16)):
+        wl = workload(name) if name != "mlp_up_int3" else workload("mlp_up", codec="int3")
         b = Bench(wl, batch, dev, torch, C)
         total, per, _ = b.timed(20000, 200, stream)
         gbs = b.bytes * 20000 / total / 1e9

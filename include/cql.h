@@ -184,7 +184,7 @@ enum {
  * (cql_workspace_init) before its next use. */
 #define CQL_FLAG_DEBUG_SKIP_X 0x100u
 /* Decode on the CUDA cores even where the tensor-core decode applies (2:4
- * int4 layers); for comparing the two designs on the same layer. */
+ * int4 and int3 layers); for comparing the two designs on the same layer. */
 #define CQL_FLAG_CUDA_CORE 0x200u
 
 /* Layer descriptor, 64 bytes, stored verbatim in the packed header. */
@@ -310,8 +310,8 @@ cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t s
  *   rounded to x_dt, exact unless a value falls into x_dt's subnormal range)
  *   into the workspace; every later step reads x'.
  *   batch     1..16 runs the decode path: sparse tcgen05 MMAs for 2:4 int4
- *             layers with fp16/bf16 x, a CUDA-core GEMV for the other codecs
- *             and masks; larger batches run the tcgen05 tensor-core prefill
+ *             and int3 layers with fp16/bf16 x, a CUDA-core GEMV for the
+ *             other codecs and masks; larger batches run the tcgen05 tensor-core prefill
  *             GEMM, which is implemented for 2:4 int4 layers (others:
  *             CQL_ERR_UNSUPPORTED).
  *   workspace device, >= cql_workspace_size bytes, 256-byte aligned, zeroed

@@ -1,5 +1,5 @@
-// Decode main term on the sparse tensor cores: 2:4 mask, int4 codes, batch
-// 1..16.  y_acc[b][n] += sum_g s[n][g] * sum_{k in g} q[n][k] x[b][k]
+// Decode main term on the sparse tensor cores: 2:4 mask, int4 or int3 codes,
+// batch 1..16.  y_acc[b][n] += sum_g s[n][g] * sum_{k in g} q[n][k] x[b][k]
 // (SLiM-Quant's per-group scale on a 2:4-pruned matrix, SLiM review summary
 // "SLIM-Quant"; the 2:4 pattern is what the sparse tensor cores execute).
 //
@@ -10,7 +10,9 @@
 //     box's 8 or 16 rows) arrives in chunks of 1024 columns, one 3-D TMA box
 //     per chunk;
 //   * a converter warpgroup (lanes = rows, as the planes are laid out) turns
-//     the 64 kept codes of each row into exact bf16/f16 integers and writes
+//     the 64 kept codes of each row (int4: 32 bytes, two slabs; int3: 24
+//     bytes inside the two slabs that cover them) into exact bf16/f16
+//     integers and writes
 //     them straight into tensor memory (compressed A, 32 columns), and writes
 //     the META codes, regrouped across lanes into the order the sparse MMA
 //     reads them, next to it;
@@ -165,6 +167,25 @@ CQL_DEV uint32_t code_pair(uint32_t lo, uint32_t hi, uint32_t sel) {
 }
 
 
+// One 2:4 group's two 3-bit codes u (bits 0..2 and 3..5 of 'six') as exact
+// 16-bit integers q = u - 4: placed at bits 0 and 16 under the exponent of
+// 128 (bf16) or 1024 (f16), then one packed subtraction of 132 (1028).
+template <bool F16>
+CQL_DEV uint32_t code_pair3(uint32_t six) {
+  const uint32_t t = (six & 7u) | ((six & 0x38u) << 13);
+  constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
+  const uint32_t a = t | magic;
+  uint32_t q;
+  if (F16) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x64046404u));    // 1028
+  else asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x43044304u));      // 132
+  return q;
+}
+
+// First 16-byte slab (of the two a converter fetches) of group g's codes in
+// a row: int4 codes take 32 bytes a group, int3 codes 24 (at byte 24 g).
+template <int BITS>
+CQL_HD uint32_t tc_code_slab(uint32_t g) { return BITS == 4 ? 2u * g : (24u * g) >> 4; }
+
 // Instruction descriptor: sparse, D f32, A = B = bf16 (or f16), K-major,
 // M = 128, N = 16.
 CQL_HD uint32_t tc_idesc(bool f16) {
@@ -299,7 +320,7 @@ CQL_DEV void tc_side_work(const DecodeParams& p, int iw, int lane, const SideFir
 
 // 88 registers per thread: 640 x 88 leaves room for one epilogue block (128
 // threads) to become resident beside this kernel and prefetch its operands.
-template <int B, bool F16>
+template <int B, bool F16, int BITS>
 __global__ void __maxnreg__(88)
     k_decode_tc(const __grid_constant__ CUtensorMap tmX, DecodeParams p, TcGeom geo) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -433,7 +454,7 @@ __global__ void __maxnreg__(88)
       const uint32_t rb = 4u * ld.rt + qq;
       uint8_t* slot = ring + slot_i * TC_SLOT_BYTES;
 #ifdef CQL_CHECKED
-      const uint32_t ov = rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
+      const uint32_t ov = rb * vstride + tc_code_slab<BITS>((uint32_t)ld.g) * 512u + lane * 16;
       const uint32_t om = rb * mstride + (uint32_t)ld.g * 512u + lane * 16;
       const uint32_t os = rb * sstride + (uint32_t)(ld.g >> 3) * 512u + lane * 16;
       if (CQL_IN(p.err, ov + 512 + 15, p.plane_len[CQL_PLANE_VALUES], 111)) {
@@ -443,7 +464,7 @@ __global__ void __maxnreg__(88)
       if (CQL_IN(p.err, om + 15, p.plane_len[CQL_PLANE_META], 112)) cp_async16(slot + 1024, p.meta + om);
       if (CQL_IN(p.err, os + 15, p.plane_len[CQL_PLANE_SCALES], 113)) cp_async16(slot + 1536, p.scales + os);
 #else
-      const uint8_t* vsrc = p.values + rb * vstride + (uint32_t)ld.g * 1024u + lane * 16;
+      const uint8_t* vsrc = p.values + rb * vstride + tc_code_slab<BITS>((uint32_t)ld.g) * 512u + lane * 16;
       cp_async16(slot, vsrc);
       cp_async16(slot + 512, vsrc + 512);
       cp_async16(slot + 1024, p.meta + rb * mstride + (uint32_t)ld.g * 512u + lane * 16);
@@ -519,12 +540,29 @@ __global__ void __maxnreg__(88)
       const uint32_t sc16 = *reinterpret_cast<const uint16_t*>(slot + 1536 + 2 * (g & 7));
       const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
       uint32_t a[32];
+      if constexpr (BITS == 4) {
 #pragma unroll
-      for (int wi = 0; wi < 8; ++wi) {
-        const uint32_t hi = vw[wi] >> 4;
+        for (int wi = 0; wi < 8; ++wi) {
+          const uint32_t hi = vw[wi] >> 4;
 #pragma unroll
-        for (int by = 0; by < 4; ++by)
-          a[4 * wi + by] = code_pair<F16>(vw[wi], hi, (uint32_t)(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12)));
+          for (int by = 0; by < 4; ++by)
+            a[4 * wi + by] = code_pair<F16>(vw[wi], hi, (uint32_t)(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12)));
+        }
+      } else {
+        // the group's 24 bytes start at byte 0 or 8 of the 32 fetched
+        // (24 g mod 16); pair m (the group's two kept codes) is stream
+        // bits [6 m, 6 m + 6)
+        const bool odd = (g & 1) != 0;
+        uint32_t ws[7];
+#pragma unroll
+        for (int k = 0; k < 6; ++k) ws[k] = odd ? vw[k + 2] : vw[k];
+        ws[6] = 0u;
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          const int wi = (6 * m) >> 5, sh = (6 * m) & 31;
+          const uint32_t six = sh <= 26 ? (ws[wi] >> sh) : __funnelshift_r(ws[wi], ws[wi + 1], sh);
+          a[m] = code_pair3<F16>(six);
+        }
       }
       // META: this row's 32-bit code word of each K step holds groups 0..7 of
       // it; the sparse MMA wants, in lane 16h + i, rows 16h + i and 16h + 8 + i
@@ -569,11 +607,11 @@ __global__ void __maxnreg__(88)
 // host launch
 // ---------------------------------------------------------------------------
 bool decode_tc_eligible(const DecodeParams& p) {
-  return p.d.mask == CQL_MASK_2_4 && p.d.codec == CQL_CODEC_INT4_SYM && p.batch >= 1 && p.batch <= 16 &&
-         (p.xdt == CQL_DT_BF16 || p.xdt == CQL_DT_F16);
+  return p.d.mask == CQL_MASK_2_4 && (p.d.codec == CQL_CODEC_INT4_SYM || p.d.codec == CQL_CODEC_INT3_SYM) &&
+         p.batch >= 1 && p.batch <= 16 && (p.xdt == CQL_DT_BF16 || p.xdt == CQL_DT_F16);
 }
 
-template <int B, bool F16>
+template <int B, bool F16, int BITS>
 static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
   TcGeom geo;
   geo.n_rt = p.d.n_out / 128;
@@ -584,7 +622,7 @@ static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
   if (!make_map_xchunk(&mx, p.x, (uint64_t)p.batch, (uint64_t)p.d.k_in, tc_xrows<B>(), 2 * TC_KC)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(TcSmem) + 1024;
   static std::atomic<uint64_t> attr_done{0};
-  cudaError_t e = ensure_smem_attr(attr_done, (const void*)k_decode_tc<B, F16>, (int)smem);
+  cudaError_t e = ensure_smem_attr(attr_done, (const void*)k_decode_tc<B, F16, BITS>, (int)smem);
   if (e != cudaSuccess) return e;
   uint64_t grid = (uint64_t)device_sm_count();
   if (grid > (uint64_t)geo.n_tiles) grid = (uint64_t)geo.n_tiles;
@@ -598,12 +636,14 @@ static cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st, bool pdl) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_decode_tc<B, F16>, mx, p, geo);
+  return cudaLaunchKernelEx(&cfg, k_decode_tc<B, F16, BITS>, mx, p, geo);
 }
 
 template <int B>
 static cudaError_t launch_tc_b(const DecodeParams& p, cudaStream_t st, bool pdl) {
-  return p.xdt == CQL_DT_F16 ? launch_tc<B, true>(p, st, pdl) : launch_tc<B, false>(p, st, pdl);
+  if (p.d.codec == CQL_CODEC_INT3_SYM)
+    return p.xdt == CQL_DT_F16 ? launch_tc<B, true, 3>(p, st, pdl) : launch_tc<B, false, 3>(p, st, pdl);
+  return p.xdt == CQL_DT_F16 ? launch_tc<B, true, 4>(p, st, pdl) : launch_tc<B, false, 4>(p, st, pdl);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int bpad, cudaStream_t st, bool pdl) {

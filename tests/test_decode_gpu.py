@@ -29,6 +29,10 @@ REDUCED = {
     # chunk), fp16 x; 16 row tiles x 33 groups = 528 tiles, so CTAs hold
     # several tiles and cross row tiles and x chunks
     "int4_2of4_csr_ragged": workload("mlp_up", n=2048, k=4224, outlier_frac=0.002, rank=48, x_dtype="f16"),
+    # int3 2:4 on the tensor cores: 24-byte code groups straddling slabs,
+    # an odd group count (the last group at byte offset 0 of its slabs), CSR
+    "int3_2of4_tc": workload("mlp_up", n=1536, k=2176, codec="int3", outlier_frac=0.001, rank=64),
+    "mlp_up_int3": workload("mlp_up", codec="int3"),
 }
 FULL = {
     "mlp_up": workload("mlp_up"),
@@ -82,6 +86,8 @@ def test_pack_bit_exact(name, cuda_dev):
     ("lut4_lr", (1, 4)),
     ("bitmap_int4_csr", (1, 9)),
     ("int4_2of4_csr_ragged", (1, 3, 8, 13)),
+    ("int3_2of4_tc", (1, 4, 9, 16)),
+    ("mlp_up_int3", (1, 16)),
     ("mlp_up", (1, 4, 16)),
     ("lut_dense_sparse", (1, 8)),
     ("down_unstructured", (1, 2, 4, 8, 16)),
@@ -210,9 +216,10 @@ def test_bounded_wait_runs_out_and_is_reported(batch, cuda_dev):
     check_close(y, case.reference(batch), "f32", what=f"after timeout B={batch}")
 
 
-@pytest.mark.parametrize("name,batches", [("mlp_up_small", (1, 4, 16)), ("int4_2of4_csr_ragged", (1, 13))])
+@pytest.mark.parametrize("name,batches", [("mlp_up_small", (1, 4, 16)), ("int4_2of4_csr_ragged", (1, 13)),
+                                          ("int3_2of4_tc", (1, 16)), ("int3_2of4", (3,))])
 def test_cuda_core_decode_of_2of4_int4(name, batches, cuda_dev):
-    """The CUDA-core decode of a 2:4 int4 layer (selected by flag; the
+    """The CUDA-core decode of a 2:4 int4 or int3 layer (selected by flag; the
     tensor-core decode is the default for these layers) against the oracle."""
     import torch
     case = get_case(name, cuda_dev)
