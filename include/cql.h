@@ -311,9 +311,11 @@ cql_status cql_workspace_init(void* workspace, uint64_t ws_bytes, cql_stream_t s
  *   into the workspace; every later step reads x'.
  *   batch     1..16 runs the decode path: sparse tcgen05 MMAs for 2:4 int4
  *             and int3 layers with fp16/bf16 x, a CUDA-core GEMV for the
- *             other codecs and masks; larger batches run the tcgen05 tensor-core prefill
- *             GEMM, which is implemented for 2:4 int4 layers (others:
- *             CQL_ERR_UNSUPPORTED).
+ *             other codecs and masks; larger batches run the tcgen05
+ *             prefill GEMM: on the sparse tensor cores for 2:4 int4 and
+ *             int3 layers, dense for int4 / int3 layers without a mask;
+ *             LUT codecs, the bitmap mask and CSR outliers give
+ *             CQL_ERR_UNSUPPORTED there.
  *   workspace device, >= cql_workspace_size bytes, 256-byte aligned, zeroed
  *             by cql_workspace_init before its first use with a given layer
  *             and batch (the forward leaves it ready for the next call with

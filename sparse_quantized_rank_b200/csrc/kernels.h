@@ -185,7 +185,7 @@ bool make_map_rowblocks(CUtensorMap* m, const void* plane, uint64_t block_bytes,
 
 // Prefill scratch (inside the forward workspace): byte offsets.
 struct PrefillLayout {
-  bool sparse;     // 2:4 int4: the sparse GEMM (weights dequantised on chip)
+  bool sparse;     // 2:4 int4 / int3: the sparse GEMM (weights dequantised on chip)
   int r3;          // adapter extension columns (3 r rounded up to 64)
   int rrows;       // R rows padded to 128
   int r_pad;       // rank rounded up to 32

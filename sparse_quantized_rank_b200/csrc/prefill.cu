@@ -390,7 +390,7 @@ PrefillLayout prefill_layout(const cql_desc& d, int m) {
   L.r3 = r ? (int)((3 * r + 63) / 64 * 64) : 0;
   L.rrows = r ? (int)((r + 127) / 128 * 128) : 0;
   L.r_pad = (int)((r + 31) / 32 * 32);
-  L.sparse = d.mask == CQL_MASK_2_4 && d.codec == CQL_CODEC_INT4_SYM;
+  L.sparse = d.mask == CQL_MASK_2_4 && (d.codec == CQL_CODEC_INT4_SYM || d.codec == CQL_CODEC_INT3_SYM);
   // the sparse GEMM dequantises the weights on chip: only the adapter
   // columns [N][r3] are staged in memory
   L.ldq = L.sparse ? L.r3 : (int)(k + L.r3);

@@ -1,4 +1,5 @@
-// Prefill main GEMM on the sparse tensor cores, 2:4 int4 layers (batch > 16):
+// Prefill main GEMM on the sparse tensor cores, 2:4 int4 and int3 layers
+// (batch > 16):
 //
 //   Y^T[n][t] = sum_g s[n][g] * (sum_{k in g} q[n][k] X[t][k])  +  L^ T^T
 //
@@ -114,7 +115,21 @@ CQL_DEV uint32_t code_pair(uint32_t lo, uint32_t hi, uint32_t sel) {
   return q;
 }
 
+// One 2:4 group's two 3-bit codes (bits 0..2 and 3..5 of 'six') as exact
+// 16-bit integers q = u - 4: placed under the exponent of 128 (bf16) or 1024
+// (f16), then one packed subtraction of 132 (1028).
 template <bool F16>
+CQL_DEV uint32_t code_pair3(uint32_t six) {
+  const uint32_t t = (six & 7u) | ((six & 0x38u) << 13);
+  constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
+  const uint32_t a = t | magic;
+  uint32_t q;
+  if (F16) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x64046404u));
+  else asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(a), "r"(0x43044304u));
+  return q;
+}
+
+template <bool F16, int BITS>
 __global__ void __launch_bounds__(SP_THREADS, 1)
     k_pf_sgemm(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL,
                const __grid_constant__ CUtensorMap tmT, SpParams p) {
@@ -229,7 +244,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       if (mg == 0 || f_tile >= my_tiles) return;
       const int item = blockIdx.x + f_tile * gridDim.x;
       const uint32_t rbk = 4u * (uint32_t)(item / p.tok_tiles) + qq;
-      const uint32_t ov = rbk * vstride + (uint32_t)f_g * 1024u + lane * 16;
+      // int4: a group's codes are two slabs (32 bytes); int3: 24 bytes at
+      // byte 24 g, inside the two slabs from (24 g) / 16 on
+      const uint32_t slab0 = BITS == 4 ? 2u * (uint32_t)f_g : (24u * (uint32_t)f_g) >> 4;
+      const uint32_t ov = rbk * vstride + slab0 * 512u + lane * 16;
       const uint32_t om = rbk * mstride + (uint32_t)f_g * 512u + lane * 16;
       const uint8_t* vsrc = p.values + ov;
       uint8_t* sl = ring + slot * SP_RAW;
@@ -262,12 +280,28 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
           const uint4 mm = *reinterpret_cast<const uint4*>(sl + 1024);
           const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
           uint32_t q[32];                           // compressed A row: 64 kept values
+          if constexpr (BITS == 4) {
 #pragma unroll
-          for (int wi = 0; wi < 8; ++wi) {
-            const uint32_t hi = vw[wi] >> 4;
+            for (int wi = 0; wi < 8; ++wi) {
+              const uint32_t hi = vw[wi] >> 4;
 #pragma unroll
-            for (int by = 0; by < 4; ++by)
-              q[4 * wi + by] = code_pair<F16>(vw[wi], hi, (uint32_t)(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12)));
+              for (int by = 0; by < 4; ++by)
+                q[4 * wi + by] = code_pair<F16>(vw[wi], hi, (uint32_t)(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12)));
+            }
+          } else {
+            // the 24 bytes start at byte 0 (even group) or 8 (odd group) of
+            // the 32 fetched; pair m is stream bits [6 m, 6 m + 6)
+            const bool odd = (j & 1) != 0;            // j: the group of this item
+            uint32_t ws[7];
+#pragma unroll
+            for (int k = 0; k < 6; ++k) ws[k] = odd ? vw[k + 2] : vw[k];
+            ws[6] = 0u;
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+              const int wi = (6 * m) >> 5, sh = (6 * m) & 31;
+              const uint32_t six = sh <= 26 ? (ws[wi] >> sh) : __funnelshift_r(ws[wi], ws[wi + 1], sh);
+              q[m] = code_pair3<F16>(six);
+            }
           }
           // META: the sparse MMA wants, in lane 16h + i, rows 16h + i and
           // 16h + 8 + i side by side (16 bits each) for groups 0..3 of a K
@@ -379,25 +413,26 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 }  // namespace
 
 // The register split above assumes 128 registers a thread at launch.
-template <bool F16>
+template <bool F16, int BITS>
 static cudaError_t check_sgemm_regs() {
   static int ok = -1;
   if (ok < 0) {
     cudaFuncAttributes a;
-    if (cudaFuncGetAttributes(&a, (const void*)k_pf_sgemm<F16>) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+    if (cudaFuncGetAttributes(&a, (const void*)k_pf_sgemm<F16, BITS>) != cudaSuccess)
+      return cudaErrorInvalidDeviceFunction;
     ok = a.numRegs == 128 ? 1 : 0;
   }
   return ok ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
-template <bool F16>
+template <bool F16, int BITS>
 static cudaError_t launch_sg(const DecodeParams& p, const uint16_t* lbuf, int r3, const uint16_t* t3, bool lowrank,
                              cudaStream_t st) {
-  cudaError_t e = check_sgemm_regs<F16>();
+  cudaError_t e = check_sgemm_regs<F16, BITS>();
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> attr_done{0};
   const size_t smem = sizeof(SpSmem) + 1024;
-  if ((e = ensure_smem_attr(attr_done, (const void*)k_pf_sgemm<F16>, (int)smem)) != cudaSuccess) return e;
+  if ((e = ensure_smem_attr(attr_done, (const void*)k_pf_sgemm<F16, BITS>, (int)smem)) != cudaSuccess) return e;
   const int N = p.d.n_out, K = p.d.k_in, m = p.batch;
   CUtensorMap mX, mL, mT;
   if (!make_map(&mX, p.x, (uint64_t)m, (uint64_t)K, (uint64_t)K, SP_BN)) return cudaErrorInvalidValue;
@@ -428,14 +463,17 @@ static cudaError_t launch_sg(const DecodeParams& p, const uint16_t* lbuf, int r3
   s.err = p.err;
   const int items = s.row_tiles * s.tok_tiles;
   const int grid = items < device_sm_count() ? items : device_sm_count();
-  k_pf_sgemm<F16><<<grid, SP_THREADS, smem, st>>>(mX, mL, mT, s);
+  k_pf_sgemm<F16, BITS><<<grid, SP_THREADS, smem, st>>>(mX, mL, mT, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pf_sgemm(const DecodeParams& p, const uint16_t* lbuf, int r3, const uint16_t* t3, bool lowrank,
                             cudaStream_t st) {
-  return p.xdt == CQL_DT_F16 ? launch_sg<true>(p, lbuf, r3, t3, lowrank, st)
-                             : launch_sg<false>(p, lbuf, r3, t3, lowrank, st);
+  if (p.d.codec == CQL_CODEC_INT3_SYM)
+    return p.xdt == CQL_DT_F16 ? launch_sg<true, 3>(p, lbuf, r3, t3, lowrank, st)
+                               : launch_sg<false, 3>(p, lbuf, r3, t3, lowrank, st);
+  return p.xdt == CQL_DT_F16 ? launch_sg<true, 4>(p, lbuf, r3, t3, lowrank, st)
+                             : launch_sg<false, 4>(p, lbuf, r3, t3, lowrank, st);
 }
 
 }  // namespace cql

@@ -20,6 +20,9 @@ CASES = {
     "pf_norank": (workload("prefill_up", n=256, k=1024, rank=0), 512),
     "pf_dense_int4": (workload("prefill_up", n=128, k=256, mask="none", rank=32), 40),
     "pf_int3_2of4": (workload("prefill_up", n=128, k=384, codec="int3", rank=48), 600),
+    # int3 2:4 on the sparse tensor cores: 24-byte code groups, an odd group
+    # count (17), a ragged token tile
+    "pf_int3_2of4_sparse": (workload("prefill_up", n=1024, k=2176, codec="int3", rank=64), 333),
     "prefill_up": (workload("prefill_up"), 2048),
     "prefill_down": (workload("prefill_down"), 2048),
 }
