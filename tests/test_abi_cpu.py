@@ -156,6 +156,28 @@ def test_call_errors_return_before_launch(lib):
     assert L.cql_get_device_status(None, None, None) == C.CQL_ERR_ARG
 
 
+def test_adapter_construction_argument_errors(lib):
+    """cql_build_adapters checks its arguments on the host, before anything
+    is launched."""
+    fake = 1 << 40
+    d0 = C.make_desc(256, 512, rank=0)
+    with pytest.raises(C.CqlError) as ei:
+        C.cql_adapter_workspace_size(d0)                 # no adapters to build
+    assert ei.value.status == C.CQL_ERR_ARG
+    d = C.make_desc(256, 512, rank=16)
+    nb = C.cql_adapter_workspace_size(d)
+    assert nb >= 256 * 512 * 4 and nb % 256 == 0
+    L = lib
+    assert L.cql_build_adapters(ctypes.byref(d), None, C.CQL_DT_F32, fake, None, fake, fake, fake, nb, None) == \
+        C.CQL_ERR_ARG
+    assert L.cql_build_adapters(ctypes.byref(d), fake, C.CQL_DT_F16, fake, None, fake, fake, fake, nb, None) == \
+        C.CQL_ERR_ARG                                    # W must be fp32 or bf16
+    assert L.cql_build_adapters(ctypes.byref(d), fake, C.CQL_DT_F32, fake + 16, None, fake, fake, fake, nb, None) == \
+        C.CQL_ERR_ALIGN
+    assert L.cql_build_adapters(ctypes.byref(d), fake, C.CQL_DT_F32, fake, None, fake, fake, fake, nb - 256, None) == \
+        C.CQL_ERR_SIZE
+
+
 def test_workspace_sizes_grow_with_batch(lib):
     d = C.make_desc(11008, 4096, rank=128)
     sizes = [C.cql_workspace_size(d, b) for b in (1, 4, 16)]

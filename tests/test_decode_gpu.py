@@ -71,7 +71,8 @@ def test_pack_bit_exact(name, cuda_dev):
     if not np.array_equal(got, ref):
         diff = np.nonzero(got != ref)[0]
         lay = O.packed_layout(case.od)
-        planes = sorted({max(i for i in range(12) if lay["off"][i] <= d and lay["len"][i] > 0) for d in diff[:1000]})
+        planes = sorted({max(i for i in range(O.NPLANES) if lay["off"][i] <= d and lay["len"][i] > 0)
+                         for d in diff[:1000]})
         raise AssertionError(f"{len(diff)} bytes differ; first at {diff[:8]}; planes {planes}")
 
 
