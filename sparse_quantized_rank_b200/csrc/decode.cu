@@ -387,24 +387,36 @@ struct UnitBitmap {
     }
     __syncwarp();
     uint32_t cb = (bo & 15u) * 8u + (bitpos & 7u);
-    constexpr uint32_t mask = (1u << BITS) - 1;
     constexpr int bias = 1 << (BITS - 1);
     float a[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) a[b] = 0.0f;
+    // Every column in turn (the same column in all lanes: no divergence, x
+    // read as a shared-memory broadcast).  Per 8 columns one 32-bit window
+    // of the row's code stream holds their <= 8 kept codes; a column's code
+    // sits at the window offset advanced by BITS per kept column before it
+    // (bit-field extract), and a pruned column contributes 0.
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      uint32_t word = f.bm[w];
-      while (word) {
-        const int t = __ffs(word) - 1;
-        word &= word - 1;
-        const uint32_t wi = cb >> 5, sh = cb & 31u;
-        const uint32_t c = __funnelshift_r(win[wi * 32 + lane], win[(wi + 1) * 32 + lane], sh) & mask;
-        cb += BITS;
-        const float q = (float)((int)c - bias);
-        const float* xc = xs + (32 * w + t) * B;
+      const uint32_t word = f.bm[w];
 #pragma unroll
-        for (int b = 0; b < B; ++b) a[b] = fmaf(q, xc[b], a[b]);
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t wi = cb >> 5, sh = cb & 31u;
+        const uint32_t win32 = __funnelshift_r(win[wi * 32 + lane], win[(wi + 1) * 32 + lane], sh);
+        uint32_t off = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint32_t bit = (word >> (8 * k + t)) & 1u;
+          uint32_t c;
+          asm("bfe.u32 %0, %1, %2, %3;" : "=r"(c) : "r"(win32), "r"(off), "n"(BITS));
+          // exact integer to float: c under the exponent of 2^23, minus 2^23 + bias
+          const float q = bit ? __uint_as_float(c | kMagic) - (8388608.0f + (float)bias) : 0.0f;
+          const float* xc = xs + (32 * w + 8 * k + t) * B;
+#pragma unroll
+          for (int b = 0; b < B; ++b) a[b] = fmaf(q, xc[b], a[b]);
+          off += bit * BITS;
+        }
+        cb += __popc((word >> (8 * k)) & 0xFFu) * BITS;
       }
     }
     const float s = f16_bits_to_f32(f.s);
