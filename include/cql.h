@@ -282,6 +282,22 @@ cql_status cql_build_adapters(const cql_desc* desc, const void* W, cql_dtype w_d
                               const float* act_absmean, float* L, float* R, void* workspace, uint64_t ws_bytes,
                               cql_stream_t stream);
 
+/* Saving and loading packed layers.  A packed buffer is self-describing:
+ * copied to the host (or to a file) and back, it needs no other state.
+ *
+ * cql_read_header: the descriptor and layout stored in the header of a HOST
+ * copy of a packed buffer (at least 512 bytes readable at 'packed_host').
+ * Returns CQL_ERR_FORMAT when the magic, the version, the descriptor's
+ * validity or the stored layout (recomputed from the descriptor) does not
+ * match, CQL_ERR_SIZE when 'bytes' is smaller than the stored total.
+ *
+ * cql_plane_checksums: CRC-32 (IEEE 802.3 polynomial, the zlib/PNG
+ * checksum) of every plane of a HOST copy, out[i] for plane i (0 for an
+ * empty plane), after the same checks as cql_read_header; for verifying a
+ * layer after saving, copying or loading it.  Host only, both. */
+cql_status cql_read_header(const void* packed_host, uint64_t bytes, cql_desc* desc_out, cql_layout* layout_out);
+cql_status cql_plane_checksums(const void* packed_host, uint64_t bytes, uint32_t out[CQL_NPLANES]);
+
 /* Workspace bytes compressed_linear_forward needs for this layer and batch.
  * Host only. */
 cql_status cql_workspace_size(const cql_desc* desc, int32_t batch, uint64_t* bytes);

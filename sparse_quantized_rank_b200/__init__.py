@@ -37,7 +37,7 @@ EXPORTED = (
     "cql_status_string", "cql_version", "cql_packed_layout", "cql_pack_workspace_size",
     "pack_compressed_weight", "cql_workspace_size", "cql_workspace_init",
     "compressed_linear_forward", "cql_get_device_status", "compressed_linear_forward_noalloc",
-    "cql_adapter_workspace_size", "cql_build_adapters",
+    "cql_adapter_workspace_size", "cql_build_adapters", "cql_read_header", "cql_plane_checksums",
 )
 
 
@@ -102,6 +102,8 @@ def lib():
                                                         ctypes.c_int, I32, P]
         L.cql_adapter_workspace_size.argtypes = [ctypes.POINTER(cql_desc), ctypes.POINTER(U64)]
         L.cql_build_adapters.argtypes = [ctypes.POINTER(cql_desc), P, ctypes.c_int, P, P, P, P, P, U64, P]
+        L.cql_read_header.argtypes = [P, U64, ctypes.POINTER(cql_desc), ctypes.POINTER(cql_layout)]
+        L.cql_plane_checksums.argtypes = [P, U64, ctypes.POINTER(ctypes.c_uint32 * CQL_NPLANES)]
         for fn in EXPORTED[2:]:
             getattr(L, fn).restype = ctypes.c_int
         _libs[_active] = L
@@ -207,6 +209,24 @@ def cql_build_adapters(desc, W, w_dt, packed, act_absmean, L, R, workspace, ws_b
     _check(lib().cql_build_adapters(ctypes.byref(desc), _ptr(W), int(w_dt), _ptr(packed), _ptr(act_absmean), _ptr(L),
                                     _ptr(R), _ptr(workspace), int(ws_bytes), _stream(stream)),
            "cql_build_adapters")
+
+
+def cql_read_header(packed_host: bytes):
+    """(cql_desc, cql_layout) stored in a host copy of a packed buffer."""
+    buf = ctypes.create_string_buffer(bytes(packed_host), len(packed_host))
+    d, lay = cql_desc(), cql_layout()
+    _check(lib().cql_read_header(ctypes.cast(buf, ctypes.c_void_p), len(packed_host), ctypes.byref(d),
+                                 ctypes.byref(lay)), "cql_read_header")
+    return d, lay
+
+
+def cql_plane_checksums(packed_host: bytes):
+    """CRC-32 of every plane of a host copy of a packed buffer."""
+    buf = ctypes.create_string_buffer(bytes(packed_host), len(packed_host))
+    out = (ctypes.c_uint32 * CQL_NPLANES)()
+    _check(lib().cql_plane_checksums(ctypes.cast(buf, ctypes.c_void_p), len(packed_host), ctypes.byref(out)),
+           "cql_plane_checksums")
+    return list(out)
 
 
 def cql_get_device_status(workspace, stream=None) -> int:

@@ -369,6 +369,53 @@ cql_status cql_build_adapters(const cql_desc* desc, const void* W, cql_dtype w_d
   return e == cudaSuccess ? CQL_OK : CQL_ERR_CUDA;
 }
 
+cql_status cql_read_header(const void* packed_host, uint64_t bytes, cql_desc* desc_out, cql_layout* layout_out) {
+  if (packed_host == nullptr || desc_out == nullptr) return CQL_ERR_ARG;
+  if (bytes < CQL_HEADER_BYTES) return CQL_ERR_SIZE;
+  const uint8_t* b = static_cast<const uint8_t*>(packed_host);
+  uint32_t ver = 0;
+  memcpy(&ver, b + 4, 4);
+  if (memcmp(b, "CQL1", 4) != 0 || ver != CQL_VERSION) return CQL_ERR_FORMAT;
+  cql_desc d;
+  memcpy(&d, b + 8, sizeof(cql_desc));
+  if (validate_desc(&d) != CQL_OK) return CQL_ERR_FORMAT;
+  cql_layout stored, expect;
+  memcpy(&stored.total_bytes, b + 72, 8);
+  memcpy(&stored.nnz, b + 80, 8);
+  memcpy(stored.off, b + 88, 8 * CQL_NPLANES);
+  memcpy(stored.len, b + 88 + 8 * CQL_NPLANES, 8 * CQL_NPLANES);
+  compute_layout(d, &expect);
+  if (stored.total_bytes != expect.total_bytes || stored.nnz != expect.nnz ||
+      memcmp(stored.off, expect.off, sizeof(expect.off)) != 0 || memcmp(stored.len, expect.len, sizeof(expect.len)) != 0)
+    return CQL_ERR_FORMAT;
+  if (bytes < stored.total_bytes) return CQL_ERR_SIZE;
+  *desc_out = d;
+  if (layout_out != nullptr) *layout_out = stored;
+  return CQL_OK;
+}
+
+cql_status cql_plane_checksums(const void* packed_host, uint64_t bytes, uint32_t out[CQL_NPLANES]) {
+  if (out == nullptr) return CQL_ERR_ARG;
+  cql_desc d;
+  cql_layout lay;
+  const cql_status s = cql_read_header(packed_host, bytes, &d, &lay);
+  if (s != CQL_OK) return s;
+  // CRC-32, reflected, polynomial 0xEDB88320, initial and final xor ~0
+  uint32_t table[256];
+  for (uint32_t i = 0; i < 256; ++i) {
+    uint32_t c = i;
+    for (int k = 0; k < 8; ++k) c = (c & 1u) ? 0xEDB88320u ^ (c >> 1) : c >> 1;
+    table[i] = c;
+  }
+  const uint8_t* b = static_cast<const uint8_t*>(packed_host);
+  for (int i = 0; i < CQL_NPLANES; ++i) {
+    uint32_t c = 0xFFFFFFFFu;
+    for (uint64_t j = 0; j < lay.len[i]; ++j) c = table[(c ^ b[lay.off[i] + j]) & 0xFFu] ^ (c >> 8);
+    out[i] = lay.len[i] ? ~c : 0u;
+  }
+  return CQL_OK;
+}
+
 cql_status cql_get_device_status(void* workspace, cql_stream_t stream, cql_status* out) {
   if (out == nullptr) return CQL_ERR_ARG;
   if (workspace == nullptr) {

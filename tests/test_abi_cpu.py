@@ -8,6 +8,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import oracle as O
@@ -183,3 +184,59 @@ def test_workspace_sizes_grow_with_batch(lib):
     sizes = [C.cql_workspace_size(d, b) for b in (1, 4, 16)]
     assert sizes[0] < sizes[1] < sizes[2]
     assert all(s % 256 == 0 for s in sizes)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict(n=128, k=256, rank=16)),
+    ("lut_dense_sparse", dict(n=128, k=256)),
+    ("mlp_up_slimo", dict(n=128, k=512, rank=16, salient_channels=5, salient_log2=1)),
+    ("down_unstructured", dict(n=128, k=384, rank=16, clip_alpha=0.0)),
+])
+def test_saved_buffer_header_and_checksums(lib, name, over):
+    """A host copy of a packed buffer (the oracle's, byte-identical to the
+    GPU packer's) gives back its descriptor and layout, and every plane's
+    CRC-32 equals zlib's."""
+    import zlib
+    from workloads import make_layer_inputs, workload
+    wl = workload(name, **over)
+    inp = make_layer_inputs(wl, max_batch=1)
+    od = O.desc_for(wl)
+    parts = O.compress(od, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
+    buf = bytes(O.pack_bytes(od, parts))
+    d, lay = C.cql_read_header(buf)
+    assert (d.n_out, d.k_in, d.mask, d.codec, d.rank) == (od.n_out, od.k_in, od.mask, od.codec, od.rank)
+    assert (d.salient_channels, d.salient_log2) == (od.salient_channels, od.salient_log2)
+    if od.clip_alpha == 0.0:                              # the searched alpha is what the header holds
+        assert d.clip_alpha == np.float32(parts["clip_alpha"])
+    ol = O.packed_layout(od)
+    assert list(lay.off) == ol["off"] and list(lay.len) == ol["len"] and lay.total_bytes == len(buf)
+    crc = C.cql_plane_checksums(buf)
+    for i in range(O.NPLANES):
+        seg = buf[ol["off"][i]: ol["off"][i] + ol["len"][i]]
+        assert crc[i] == (zlib.crc32(seg) if ol["len"][i] else 0), i
+
+
+def test_saved_buffer_corruption_is_reported(lib):
+    from workloads import make_layer_inputs, workload
+    wl = workload("tiny", n=128, k=256, rank=16)
+    inp = make_layer_inputs(wl, max_batch=1)
+    od = O.desc_for(wl)
+    buf = bytearray(O.pack_bytes(od, O.compress(od, inp["w"], inp["L"], inp["R"])))
+
+    def status(b):
+        try:
+            C.cql_read_header(bytes(b))
+            return C.CQL_OK
+        except C.CqlError as e:
+            return e.status
+    assert status(buf) == C.CQL_OK
+    assert status(buf[:-256]) == C.CQL_ERR_SIZE           # truncated
+    assert status(buf[:100]) == C.CQL_ERR_SIZE            # not even a header
+    bad = bytearray(buf); bad[0] ^= 1                     # magic
+    assert status(bad) == C.CQL_ERR_FORMAT
+    bad = bytearray(buf); bad[4] ^= 1                     # version
+    assert status(bad) == C.CQL_ERR_FORMAT
+    bad = bytearray(buf); bad[8] ^= 1                     # n_out no longer a multiple of 128
+    assert status(bad) == C.CQL_ERR_FORMAT
+    bad = bytearray(buf); bad[88 + 8 * 13 + 8] ^= 1       # a stored plane length
+    assert status(bad) == C.CQL_ERR_FORMAT
