@@ -44,7 +44,7 @@
  * PACKED FORMAT (version 2)
  * ------------------------------------------------------------------------
  * A packed weight is one contiguous device buffer: a 512-byte header followed
- * by up to 12 planes, in the order of the CQL_PLANE_* indices.  Every plane
+ * by up to 13 planes, in the order of the CQL_PLANE_* indices.  Every plane
  * starts on a 256-byte boundary; an absent plane has length 0 and the offset
  * where it would start.  All multi-byte fields are little-endian.
  *
@@ -243,7 +243,12 @@ cql_status cql_pack_workspace_size(const cql_desc* desc, uint64_t* bytes);
  *   packed    device, >= cql_layout.total_bytes, 256-byte aligned; every byte
  *             of it is written.
  *   workspace device scratch of >= cql_pack_workspace_size bytes, 256-byte
- *             aligned; its contents on entry do not matter.
+ *             aligned; its contents on entry do not matter.  Its first 8
+ *             bytes are an error word that the pack clears first and that
+ *             only the range-checked library (libcql_checked) ever sets:
+ *             CQL_ERR_RANGE when a pack kernel's index fell outside its
+ *             plane.  Read it with cql_get_device_status(workspace, ...)
+ *             before reusing the workspace.
  * The result is bit-exact with the CPU oracle on every byte.  Inputs must be
  * finite. */
 cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype w_dt,
@@ -366,7 +371,9 @@ cql_status compressed_linear_forward_noalloc(const cql_desc* desc, const void* p
  * workspace: *out = CQL_OK or the cql_status a kernel recorded.  After an
  * error the rest of the workspace is in an undefined state: initialise it
  * again with cql_workspace_init before the next forward that uses it.
- *   workspace  a forward workspace, or NULL for the fixed scratch array of
+ *   workspace  a forward workspace, a pack workspace (after
+ *              pack_compressed_weight: CQL_OK, or CQL_ERR_RANGE from the
+ *              range-checked library), or NULL for the fixed scratch array of
  *              compressed_linear_forward_noalloc on the current device (each
  *              no-workspace call clears that word when it starts, so this
  *              reports the most recent such call; CQL_OK if none ran). */

@@ -327,3 +327,9 @@ class CompressedLinear:
     def device_status(self, batch: int, stream=None) -> int:
         ws, _ = self.workspace(batch, stream)
         return cql_get_device_status(ws, stream)
+
+    def pack_status(self, stream=None) -> int:
+        """Device error word of the pack that built this layer: CQL_OK, or
+        CQL_ERR_RANGE when the range-checked library saw a pack kernel index
+        outside its plane."""
+        return cql_get_device_status(self._pack_ws, stream)

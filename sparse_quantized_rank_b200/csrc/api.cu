@@ -128,6 +128,7 @@ PackWorkspace pack_workspace_layout(const cql_desc& d) {
   const uint64_t total = (uint64_t)d.n_out * d.k_in;
   const uint64_t nblk = (total + kTopkChunk - 1) / kTopkChunk;
   uint64_t pos = 0;
+  w.err = pos;       pos = align256(pos + 8);       // device error word (read by cql_get_device_status)
   w.out_bits = pos;  pos = align256(pos + (d.outlier_frac > 0.0f ? total / 8 : 0));
   w.state = pos;     pos = align256(pos + sizeof(TopkState));
   w.hist = pos;      pos = align256(pos + 256 * 4);
@@ -245,6 +246,8 @@ cql_status pack_compressed_weight(const cql_desc* desc, const void* W, cql_dtype
   p.l_values = base + lay.off[CQL_PLANE_L_VALUES];
   p.l_scales = reinterpret_cast<uint16_t*>(base + lay.off[CQL_PLANE_L_SCALES]);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.err = reinterpret_cast<uint32_t*>(ws + pw.err);
+  for (int i = 0; i < CQL_NPLANES; ++i) p.plane_len[i] = lay.len[i];
   p.out_bits = reinterpret_cast<uint32_t*>(ws + pw.out_bits);
   p.topk_state = reinterpret_cast<TopkState*>(ws + pw.state);
   p.topk_hist = reinterpret_cast<uint32_t*>(ws + pw.hist);

@@ -58,10 +58,13 @@ struct PackParams {
   float* alpha_dev;                  // the searched alpha (device), or null: use 'alpha'
   unsigned long long* alpha_hist;    // [1024] histogram
   const float* fisher;               // [N*K] Fisher diagonal (LUT codecs), or null
+  // range checks (checked build): error word, plane lengths in bytes
+  uint32_t* err;                     // first word of the pack workspace
+  uint64_t plane_len[CQL_NPLANES];
 };
 
 struct PackWorkspace {
-  uint64_t out_bits, state, hist, tiecnt, tieoff, row_counts, w_scaled, sal_partial, sal, sal_flag, alpha, total;
+  uint64_t err, out_bits, state, hist, tiecnt, tieoff, row_counts, w_scaled, sal_partial, sal, sal_flag, alpha, total;
 };
 PackWorkspace pack_workspace_layout(const cql_desc& d);
 

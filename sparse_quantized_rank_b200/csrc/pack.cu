@@ -33,6 +33,15 @@ CQL_DEV uint32_t lanemask_lt() {
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
 }
+// Range check of an access of `width` bytes at byte j of row i of a
+// row-interleaved packed plane: j inside the row and the byte offset inside
+// the plane.  Checked build only (CQL_ERR_RANGE with the site, access
+// skipped); the constant true otherwise.
+CQL_DEV bool plane_in(const PackParams& p, uint64_t i, uint64_t j, uint64_t row_bytes, uint64_t width, int plane,
+                      uint32_t site) {
+  return CQL_IN(p.err, j + width - 1, row_bytes, site) &&
+         CQL_IN(p.err, rit(i, j, row_bytes) + width - 1, p.plane_len[plane], site);
+}
 // Symmetric RTN code: clamp(rint(w / s), -qmax, qmax), 0 when s == 0.
 CQL_DEV int rtn_code(double w, double s, int qmax) {
   if (!(s > 0.0)) return 0;
@@ -149,7 +158,7 @@ CQL_DEV uint32_t block_rank256(bool flag, uint32_t* ws, uint32_t* total) {
 
 __global__ void __launch_bounds__(256) k_topk_mark(const void* W, int wdt, uint64_t total,
                                                    const TopkState* st, const uint32_t* tieoff,
-                                                   uint32_t* out_bits) {
+                                                   uint32_t* out_bits, uint32_t* err) {
   __shared__ uint32_t ws[8];
   const uint32_t T = st->prefix, want = st->want;
   uint32_t running = tieoff[blockIdx.x];
@@ -165,17 +174,20 @@ __global__ void __launch_bounds__(256) k_topk_mark(const void* W, int wdt, uint6
     const bool sel = gt || (eq && rank < want);
     const uint32_t word = __ballot_sync(0xffffffffu, sel);
     const uint64_t w0 = chunk + (threadIdx.x & ~31u);
-    if ((threadIdx.x & 31) == 0 && w0 < end) out_bits[w0 >> 5] = word;
+    if ((threadIdx.x & 31) == 0 && w0 < end && CQL_IN(err, w0 >> 5, total / 32, 501)) out_bits[w0 >> 5] = word;
     running += tot;
   }
 }
 
 // Outliers per row (warp per row) -> counts.
-__global__ void k_row_popcount(const uint32_t* bits, int n_rows, int words_per_row, uint32_t* counts) {
+__global__ void k_row_popcount(const uint32_t* bits, int n_rows, int words_per_row, uint32_t* counts, uint32_t* err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= n_rows) return;
   uint32_t c = 0;
-  for (int w = lane; w < words_per_row; w += 32) c += __popc(bits[(uint64_t)warp * words_per_row + w]);
+  for (int w = lane; w < words_per_row; w += 32) {
+    const uint64_t i = (uint64_t)warp * words_per_row + w;
+    if (CQL_IN(err, i, (uint64_t)n_rows * words_per_row, 502)) c += __popc(bits[i]);
+  }
   for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if (lane == 0) counts[warp] = c;
 }
@@ -224,7 +236,7 @@ __global__ void __launch_bounds__(256) k_mask_bitmap(PackParams p) {
     const bool keep = gt || (eq && rank < want);
     const uint32_t word = __ballot_sync(0xffffffffu, keep);
     const int c0 = chunk + (t & ~31);
-    if ((t & 31) == 0 && c0 < K)
+    if ((t & 31) == 0 && c0 < K && plane_in(p, n, (uint64_t)c0 / 8, p.rb.meta, 4, CQL_PLANE_META, 503))
       *reinterpret_cast<uint32_t*>(p.meta + rit(n, (uint64_t)c0 / 8, p.rb.meta)) = word;
     running += tot;
   }
@@ -269,7 +281,8 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
   constexpr int qmax = (1 << (BITS - 1)) - 1;
   const bool has_csr = p.out_bits != nullptr;
   const double alpha = p.alpha_dev != nullptr ? (double)*p.alpha_dev : p.alpha;   // searched or given
-  uint32_t kept_run = 0, out_run = has_csr ? (uint32_t)p.csr_rowptr[n] : 0u;
+  uint32_t kept_run = 0, out_run = 0;
+  if (has_csr && CQL_IN(p.err, 4ull * n + 3, p.plane_len[CQL_PLANE_CSR_ROWPTR], 511)) out_run = (uint32_t)p.csr_rowptr[n];
   for (int g = 0; g < K / kGroup; ++g) {
     const int c = g * kGroup + t;
     const uint64_t idx = (uint64_t)n * K + c;
@@ -292,7 +305,8 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
       const int i0 = __ffs(m4) - 1, i1 = 31 - __clz(m4);
       pat = i0 | (i1 << 2);
     } else if (MASK == CQL_MASK_BITMAP50) {
-      keep = (p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u;
+      keep = plane_in(p, n, (uint64_t)c / 8, p.rb.meta, 1, CQL_PLANE_META, 504) &&
+             ((p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u);
     }
     // group amax over non-outliers
     float a = outl ? 0.0f : fabsf(wv);
@@ -315,15 +329,19 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
       ooff += w < warp ? s_o[w] : 0u;
       otot += s_o[w];
     }
-    if (keep) codes[kept_run + koff + __popc(kb & lanemask_lt())] = (uint8_t)(q + (1 << (BITS - 1)));
-    if (MASK == CQL_MASK_2_4 && (lane & 3) == 0) nib[c >> 2] = (uint8_t)pat;
+    const uint32_t kpos = kept_run + koff + __popc(kb & lanemask_lt());
+    if (keep && CQL_IN(p.err, kpos, K, 505)) codes[kpos] = (uint8_t)(q + (1 << (BITS - 1)));
+    if (MASK == CQL_MASK_2_4 && (lane & 3) == 0 && CQL_IN(p.err, c >> 2, K / 4, 522)) nib[c >> 2] = (uint8_t)pat;
     if (t == 0) {
-      *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * g, p.rb.scales)) = s16;
-      if (MASK == CQL_MASK_BITMAP50)
+      if (plane_in(p, n, 2 * g, p.rb.scales, 2, CQL_PLANE_SCALES, 506))
+        *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * g, p.rb.scales)) = s16;
+      if (MASK == CQL_MASK_BITMAP50 && plane_in(p, n, 2 * g, p.rb.voff, 2, CQL_PLANE_VOFF, 507))
         *reinterpret_cast<uint16_t*>(p.voff + rit(n, 2 * g, p.rb.voff)) = (uint16_t)kept_run;
     }
     const uint32_t opos = out_run + ooff + __popc(ob & lanemask_lt());
-    if (has_csr && outl && opos < p.nnz_target) {   // the selection marks exactly nnz entries
+    if (has_csr && outl && opos < p.nnz_target &&   // the selection marks exactly nnz entries
+        CQL_IN(p.err, 2ull * opos + 1, p.plane_len[CQL_PLANE_CSR_COL], 508) &&
+        CQL_IN(p.err, 2ull * opos + 1, p.plane_len[CQL_PLANE_CSR_VAL], 508)) {
       const uint32_t pos = opos;
       const double dense = keep ? __dmul_rn((double)q, s) : 0.0;
       p.csr_col[pos] = (uint16_t)c;
@@ -334,11 +352,14 @@ __global__ void __launch_bounds__(128, 1) k_codec_uniform(PackParams p) {
     __syncthreads();
   }
   const uint32_t rbv = p.rb.values;
-  for (uint32_t j = t; j < rbv; j += 128) p.values[rit(n, j, rbv)] = (uint8_t)stream_byte<BITS>(codes, kept_run, j);
+  for (uint32_t j = t; j < rbv; j += 128)
+    if (plane_in(p, n, j, rbv, 1, CQL_PLANE_VALUES, 509))
+      p.values[rit(n, j, rbv)] = (uint8_t)stream_byte<BITS>(codes, kept_run, j);
   if (MASK == CQL_MASK_2_4) {
     const uint32_t rbm = p.rb.meta;
     for (uint32_t j = t; j < rbm; j += 128)
-      p.meta[rit(n, j, rbm)] = (uint8_t)((nib[2 * j] & 15u) | ((nib[2 * j + 1] & 15u) << 4));
+      if (plane_in(p, n, j, rbm, 1, CQL_PLANE_META, 510) && CQL_IN(p.err, 2 * j + 1, K / 4, 522))
+        p.meta[rit(n, j, rbm)] = (uint8_t)((nib[2 * j] & 15u) | ((nib[2 * j + 1] & 15u) << 4));
   }
 }
 
@@ -377,7 +398,8 @@ __global__ void __launch_bounds__(128) k_alpha_hist(PackParams p, unsigned long 
       }
       keep = rank < 2;
     } else if (MASK == CQL_MASK_BITMAP50) {
-      keep = (p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u;
+      keep = plane_in(p, n, (uint64_t)c / 8, p.rb.meta, 1, CQL_PLANE_META, 512) &&
+             ((p.meta[rit(n, (uint64_t)c / 8, p.rb.meta)] >> (c & 7)) & 1u);
     }
     float a = outl ? 0.0f : fabsf(wv);
     for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -485,7 +507,8 @@ __global__ void __launch_bounds__(256, 1) k_codec_lut(PackParams p) {
     c = __dadd_rn(c, 0.0);                                    // -0 -> +0
     const uint16_t b = f64_to_f16_bits(c);
     cent[t] = f16_to_f64(b);
-    if (p.fisher == nullptr) *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
+    if (p.fisher == nullptr && plane_in(p, n, 2 * t, p.rb.scales, 2, CQL_PLANE_SCALES, 513))
+      *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
   }
   __syncthreads();
   if (p.fisher != nullptr) {
@@ -528,12 +551,14 @@ __global__ void __launch_bounds__(256, 1) k_codec_lut(PackParams p) {
     if (t < NC) {
       const uint16_t b = f64_to_f16_bits(__dadd_rn(cent[t], 0.0));
       cent[t] = f16_to_f64(b);
-      *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
+      if (plane_in(p, n, 2 * t, p.rb.scales, 2, CQL_PLANE_SCALES, 513))
+        *reinterpret_cast<uint16_t*>(p.scales + rit(n, 2 * t, p.rb.scales)) = b;
     }
     __syncthreads();
   }
   const bool has_csr = p.out_bits != nullptr;
-  uint32_t out_run = has_csr ? (uint32_t)p.csr_rowptr[n] : 0u;
+  uint32_t out_run = 0;
+  if (has_csr && CQL_IN(p.err, 4ull * n + 3, p.plane_len[CQL_PLANE_CSR_ROWPTR], 511)) out_run = (uint32_t)p.csr_rowptr[n];
   for (int chunk = 0; chunk < K; chunk += 256) {
     const int c = chunk + t;
     uint32_t code = 0;
@@ -552,7 +577,9 @@ __global__ void __launch_bounds__(256, 1) k_codec_lut(PackParams p) {
     }
     uint32_t tot;
     const uint32_t r = block_rank256(o, ws, &tot);
-    if (has_csr && o && out_run + r < p.nnz_target) {
+    if (has_csr && o && out_run + r < p.nnz_target &&
+        CQL_IN(p.err, 2ull * (out_run + r) + 1, p.plane_len[CQL_PLANE_CSR_COL], 514) &&
+        CQL_IN(p.err, 2ull * (out_run + r) + 1, p.plane_len[CQL_PLANE_CSR_VAL], 514)) {
       const uint32_t pos = out_run + r;
       p.csr_col[pos] = (uint16_t)c;
       p.csr_val[pos] = f64_to_f16_bits(__dsub_rn(wv, cent[code]));
@@ -561,7 +588,8 @@ __global__ void __launch_bounds__(256, 1) k_codec_lut(PackParams p) {
   }
   __syncthreads();
   const uint32_t rbv = p.rb.values;
-  for (uint32_t j = t; j < rbv; j += 256) p.values[rit(n, j, rbv)] = (uint8_t)stream_byte<BITS>(codes, K, j);
+  for (uint32_t j = t; j < rbv; j += 256)
+    if (plane_in(p, n, j, rbv, 1, CQL_PLANE_VALUES, 515)) p.values[rit(n, j, rbv)] = (uint8_t)stream_byte<BITS>(codes, K, j);
 }
 
 // ---------------------------------------------------------------------------
@@ -580,9 +608,11 @@ __global__ void k_adapter_R(PackParams p) {
   const double s = f16_to_f64(s16);
   for (int i = 0; i < kGroup / 2; ++i) {
     const int q0 = rtn_code((double)v[2 * i], s, 7), q1 = rtn_code((double)v[2 * i + 1], s, 7);
-    p.r_values[rit(j, (uint64_t)g * 64 + i, p.rb.r_values)] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
+    if (plane_in(p, j, (uint64_t)g * 64 + i, p.rb.r_values, 1, CQL_PLANE_R_VALUES, 517))
+      p.r_values[rit(j, (uint64_t)g * 64 + i, p.rb.r_values)] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
   }
-  *reinterpret_cast<uint16_t*>(p.r_scales + rit(j, 2 * g, p.rb.r_scales)) = s16;
+  if (plane_in(p, j, 2 * g, p.rb.r_scales, 2, CQL_PLANE_R_SCALES, 518))
+    *reinterpret_cast<uint16_t*>(p.r_scales + rit(j, 2 * g, p.rb.r_scales)) = s16;
 }
 
 // L [N][r]: thread per (row group g along N, column pair jp).
@@ -597,14 +627,16 @@ __global__ void k_adapter_L(PackParams p) {
     float amax = 0.0f;
     for (int i = 0; i < kGroup; ++i) amax = fmaxf(amax, fabsf(p.L[(uint64_t)(g * kGroup + i) * r + j]));
     const uint16_t s16 = f64_to_f16_bits(__ddiv_rn((double)amax, 7.0));
-    p.l_scales[(uint64_t)g * r + j] = s16;
+    if (CQL_IN(p.err, 2 * ((uint64_t)g * r + j) + 1, p.plane_len[CQL_PLANE_L_SCALES], 519))
+      p.l_scales[(uint64_t)g * r + j] = s16;
     s[h] = f16_to_f64(s16);
   }
   for (int i = 0; i < kGroup; ++i) {
     const uint64_t row = (uint64_t)g * kGroup + i;
     const int q0 = rtn_code((double)p.L[row * r + 2 * jp], s[0], 7);
     const int q1 = rtn_code((double)p.L[row * r + 2 * jp + 1], s[1], 7);
-    p.l_values[rit(row, jp, p.rb.l_values)] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
+    if (plane_in(p, row, jp, p.rb.l_values, 1, CQL_PLANE_L_VALUES, 520))
+      p.l_values[rit(row, jp, p.rb.l_values)] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
   }
 }
 
@@ -629,6 +661,7 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
   const int N = p.d.n_out, K = p.d.k_in;
   cudaError_t e = cudaMemsetAsync(p.packed, 0, total_bytes, st);
   if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.err, 0, 8, st)) != cudaSuccess) return e;
   k_write_header<<<1, 64, 0, st>>>(hdr, p.packed);
   if (p.d.salient_channels > 0 && (e = launch_salient_pack(p, st)) != cudaSuccess) return e;
 
@@ -642,8 +675,8 @@ cudaError_t launch_pack(const PackParams& p0, const HeaderBytes& hdr, uint64_t t
     const int nblk = (int)((total + kTopkChunk - 1) / kTopkChunk);
     k_topk_tiecount<<<nblk, 256, 0, st>>>(p.W, p.wdt, total, p.topk_state, p.topk_tiecnt);
     k_scan_excl<<<1, 1024, 0, st>>>(p.topk_tiecnt, p.topk_tieoff, nblk);
-    k_topk_mark<<<nblk, 256, 0, st>>>(p.W, p.wdt, total, p.topk_state, p.topk_tieoff, p.out_bits);
-    k_row_popcount<<<(N * 32 + 255) / 256, 256, 0, st>>>(p.out_bits, N, K / 32, p.row_counts);
+    k_topk_mark<<<nblk, 256, 0, st>>>(p.W, p.wdt, total, p.topk_state, p.topk_tieoff, p.out_bits, p.err);
+    k_row_popcount<<<(N * 32 + 255) / 256, 256, 0, st>>>(p.out_bits, N, K / 32, p.row_counts, p.err);
     k_scan_excl<<<1, 1024, 0, st>>>(p.row_counts, reinterpret_cast<uint32_t*>(p.csr_rowptr), N);
   } else {
     p.out_bits = nullptr;

@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(256) k_sal_rank(const double* sal, int K, int 
 }
 
 // one block of 1024 threads: thread t owns columns [t * per, (t + 1) * per)
-__global__ void __launch_bounds__(1024) k_sal_compact(const uint8_t* flag, int K, uint16_t* list) {
+__global__ void __launch_bounds__(1024) k_sal_compact(const uint8_t* flag, int K, int m, uint16_t* list,
+                                                      uint32_t* err) {
   __shared__ int cnt[1024];
   const int per = (K + 1023) / 1024;
   const int c0 = min(K, threadIdx.x * per), c1 = min(K, c0 + per);
@@ -91,7 +92,10 @@ __global__ void __launch_bounds__(1024) k_sal_compact(const uint8_t* flag, int K
   }
   int pos = cnt[threadIdx.x] - n;
   for (int c = c0; c < c1; ++c)
-    if (flag[c]) list[pos++] = (uint16_t)c;
+    if (flag[c]) {
+      if (CQL_IN(err, pos, m, 521)) list[pos] = (uint16_t)c;
+      ++pos;
+    }
 }
 
 __global__ void __launch_bounds__(256) k_sal_scale_w(const void* W, int wdt, uint64_t total, int K,
@@ -155,7 +159,7 @@ cudaError_t launch_salient_pack(PackParams& p, cudaStream_t st) {
   k_sal_partial<<<dim3((K + 255) / 256, nblk), 256, 0, st>>>(p.W, p.wdt, K, p.sal_partial);
   k_sal_total<<<(K + 255) / 256, 256, 0, st>>>(p.sal_partial, nblk, K, p.act_absmean, p.sal);
   k_sal_rank<<<(K + 255) / 256, 256, 0, st>>>(p.sal, K, m, p.sal_flag);
-  k_sal_compact<<<1, 1024, 0, st>>>(p.sal_flag, K, p.salient);
+  k_sal_compact<<<1, 1024, 0, st>>>(p.sal_flag, K, m, p.salient, p.err);
   const uint64_t total = (uint64_t)N * K;
   const float factor = ldexpf(1.0f, p.d.salient_log2);
   const uint64_t nb = (total + 255) / 256;

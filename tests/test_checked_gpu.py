@@ -1,13 +1,16 @@
 """Parity under the range-checked build (libcql_checked.so, -DCQL_CHECKED).
 
 Every plane read, activation read, workspace access and output store of the
-forward kernels checks its index against its buffer; an index outside
+forward kernels, and every plane store of the pack kernels, checks its index
+against its buffer; an index outside
 records CQL_ERR_RANGE (with the site) and skips the access.  With a memory
 checker unavailable, this is the library's own guard against out-of-bounds
 indexing: these cases run every forward path (tensor-core decode with CSR
 and ragged shapes, the CUDA-core codecs and masks, the sparse prefill with a
-ragged token tile, SLiM^O, the no-workspace entry point) and require both a
-clean error word and parity with the oracle.
+ragged token tile, SLiM^O, the no-workspace entry point) and every packer
+path (top-k outliers, both masks, the clip search, quantile and Fisher LUTs,
+the salient channel list, adapters), and require clean error words, packed
+bytes equal to the oracle's and parity with the oracle.
 """
 import ctypes
 
@@ -28,6 +31,12 @@ CASES = {
     "int4_dense_csr": (workload("mlp_up", n=256, k=640, mask="none", outlier_frac=0.003, rank=16), (1, 6)),
     "prefill_small": (workload("prefill_up", n=256, k=512, rank=64), (300,)),
     "slimo_small": (workload("mlp_up_slimo", n=1024, k=1024, rank=32, salient_channels=10), (1, 5, 40)),
+    # packer paths the cases above do not reach: the clip search (2:4 and
+    # bitmap), bitmap int4 with CSR outliers, Fisher k-means LUT4
+    "alpha_2of4": (workload("mlp_up", n=512, k=1024, clip_alpha=0.0), (1,)),
+    "alpha_bitmap_csr": (workload("down_unstructured", n=256, k=768, codec="int4", outlier_frac=0.002,
+                                  clip_alpha=0.0), (1, 4)),
+    "fisher_lut4": (workload("lut_dense_sparse", n=256, k=512, codec="lut4", fisher=True), (1, 2)),
 }
 
 
@@ -43,6 +52,10 @@ def test_checked_build_parity(name, checked_lib, cuda_dev):
     import torch
     wl, batches = CASES[name]
     case = Case(wl, cuda_dev, max_batch=max(batches))
+    # the pack ran under the checked library too: clean error word, every
+    # byte equal to the oracle's
+    assert case.layer.pack_status() == C.CQL_OK, f"{name}: checked build recorded an error in the pack"
+    assert (case.packed_bytes() == case.ref_bytes).all(), f"{name}: packed bytes differ from the oracle's"
     for b in batches:
         y = case.forward(b, torch.float32)
         torch.cuda.synchronize()
