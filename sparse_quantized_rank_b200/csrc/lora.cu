@@ -420,13 +420,16 @@ LoraWorkspace lora_workspace_layout(const cql_desc& d) {
 }
 
 // X [rows][p] -> orthonormal columns (CholeskyQR, twice), result in X
-static void orthonormalise(float* X, float* tmp, int rows, int p, double* G, double* U, double* Ri, cudaStream_t st) {
+static cudaError_t orthonormalise(float* X, float* tmp, int rows, int p, double* G, double* U, double* Ri,
+                                  cudaStream_t st) {
   for (int round = 0; round < 2; ++round) {
     k_lr_gram<<<dim3(p / 32, p / 32), dim3(32, 32), 0, st>>>(X, rows, p, G);
     k_lr_chol<<<1, 1024, 0, st>>>(G, p, U, Ri);
     k_lr_apply<<<blocks_for((uint64_t)rows * p, 256), 256, 0, st>>>(X, rows, p, Ri, tmp);
-    cudaMemcpyAsync(X, tmp, (size_t)rows * p * 4, cudaMemcpyDeviceToDevice, st);
+    const cudaError_t e = cudaMemcpyAsync(X, tmp, (size_t)rows * p * 4, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
   }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_build_adapters(const DecodeParams& p, const void* W, int wdt, const float* act,
@@ -457,13 +460,14 @@ cudaError_t launch_build_adapters(const DecodeParams& p, const void* W, int wdt,
   k_lr_rand<<<1184, 256, 0, st>>>((uint64_t)K * P, Z);
   // Y = Es Omega; Q = orth(Y)
   k_lr_gemm<false><<<dim3(P / 32, N / 64), 256, 0, st>>>(Es, N, K, Z, P, Y);
-  orthonormalise(Y, Y2, N, P, G, U, Ri, st);
-  for (int it = 0; it < kLrIters; ++it) {
+  cudaError_t e = orthonormalise(Y, Y2, N, P, G, U, Ri, st);
+  for (int it = 0; it < kLrIters && e == cudaSuccess; ++it) {
     k_lr_gemm<true><<<dim3(P / 32, K / 64), 256, 0, st>>>(Es, N, K, Y, P, Z);
-    orthonormalise(Z, Z2, K, P, G, U, Ri, st);
+    if ((e = orthonormalise(Z, Z2, K, P, G, U, Ri, st)) != cudaSuccess) break;
     k_lr_gemm<false><<<dim3(P / 32, N / 64), 256, 0, st>>>(Es, N, K, Z, P, Y);
-    orthonormalise(Y, Y2, N, P, G, U, Ri, st);
+    e = orthonormalise(Y, Y2, N, P, G, U, Ri, st);
   }
+  if (e != cudaSuccess) return e;
   // Z = Es^T Q (= B^T, B = Q^T Es); C = Z^T Z = B B^T
   k_lr_gemm<true><<<dim3(P / 32, K / 64), 256, 0, st>>>(Es, N, K, Y, P, Z);
   k_lr_gram<<<dim3(P / 32, P / 32), dim3(32, 32), 0, st>>>(Z, K, P, G);
