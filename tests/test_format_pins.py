@@ -175,3 +175,60 @@ def test_handworked_fixture():
         s0 = u16(buf[off[3]:], i, 0, 16)
         assert s0 == int(g["scale_fp16_bits"], 16)
         assert not any(buf[off[3] + rit_addr(i, j, 16)] for j in range(2, 16))
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict(n=128, k=256, rank=16, outlier_frac=0.003)),                 # 2:4 int4 + CSR
+    ("down_unstructured", dict(n=128, k=384, rank=0)),                         # bitmap int3
+    ("lut_dense_sparse", dict(n=128, k=256)),                                  # LUT3 + CSR
+    ("mlp_up_slimo", dict(n=128, k=512, rank=16, salient_channels=5, salient_log2=2)),
+])
+def test_compressed_matrix_is_what_the_bytes_hold(name, over):
+    """W_C (the codes' values plus the CSR outliers, in the space the codec
+    encoded), which the adapter construction compensates, equals a
+    reconstruction of each weight read field by field from the packed bytes:
+    its code (at its rank among the row's kept columns), its group scale or
+    row centroid, and its CSR entry if it has one."""
+    wl = workload(name, **over)
+    inp = make_layer_inputs(wl, max_batch=1)
+    d = O.desc_for(wl)
+    parts = O.compress(d, inp["w"], inp["L"], inp["R"], inp["act_absmean"])
+    buf = O.pack_bytes(d, parts)
+    _, _, _, _, off, ln = parse_header(buf)
+    plane = lambda p: buf[off[p]: off[p] + ln[p]]
+    n, k = d.n_out, d.k_in
+    bits = {0: 4, 1: 3, 2: 3, 3: 4}[d.codec]
+    vals, sc = plane(O.P_VALUES), plane(O.P_SCALES)
+    vrb, srb = ln[O.P_VALUES] // n, ln[O.P_SCALES] // n
+    csr = {}
+    if ln[O.P_CSR_COL]:
+        rp = np.frombuffer(bytes(plane(O.P_CSR_ROWPTR)), dtype="<i4")
+        col = np.frombuffer(bytes(plane(O.P_CSR_COL)), dtype="<u2")
+        val = np.frombuffer(bytes(plane(O.P_CSR_VAL)), dtype="<f2")
+        for i in range(n):
+            for e in range(rp[i], rp[i + 1]):
+                csr[(i, int(col[e]))] = float(val[e])
+    wc = O.compressed_matrix(parts)
+    for i in range(0, n, 9):
+        if d.mask == O.MASK_2_4:
+            meta = plane(O.P_META)
+            kept = []
+            for g in range(k // 4):
+                nib = read_bits(meta, i, k // 8, 4 * g, 4)
+                kept += [4 * g + (nib & 3), 4 * g + (nib >> 2)]
+        elif d.mask == O.MASK_BITMAP50:
+            meta = plane(O.P_META)
+            kept = [c for c in range(k) if read_bits(meta, i, k // 8, c, 1)]
+        else:
+            kept = list(range(k))
+        slot = {c: j for j, c in enumerate(kept)}
+        for c in range(k):
+            v = 0.0
+            if c in slot:
+                u = read_bits(vals, i, vrb, bits * slot[c], bits)
+                if d.codec in (O.CODEC_INT4, O.CODEC_INT3):
+                    v = (u - (1 << (bits - 1))) * f16(u16(sc, i, 2 * (c // 128), srb))
+                else:
+                    v = f16(u16(sc, i, 2 * u, srb))
+            v += csr.get((i, c), 0.0)
+            assert wc[i, c] == v, (i, c)

@@ -515,6 +515,35 @@ def test_salient_selection_brute_force_with_ties():
     assert 3 in got and 9 not in got
 
 
+def test_saliency_values_and_summation_order():
+    """Column sums of |w| times the statistic, in the fixed order the format
+    states (blocks of 64 rows, each from its first row, then the blocks in
+    order).  Integer weights give the exact value by rational arithmetic;
+    one column is built so that any other order gives another fp64 result:
+    2^53 then 63 ones in block 0 (each +1 rounds away: ties to even), then
+    64 ones in block 1, so the fixed order gives exactly 2^53 + 64 where a
+    sum of the ones first (or pairwise) gives 2^53 + 128."""
+    rng = np.random.default_rng(11)
+    n, k = 128, 24
+    w = rng.integers(-9, 10, size=(n, k)).astype(np.float64)
+    act = np.array([(c % 7 + 1) / 8.0 for c in range(k)], dtype=np.float32)
+    sal = O.channel_saliency(w, act)
+    for c in range(k):
+        exact = Fraction(float(act[c])) * sum(Fraction(abs(int(v))) for v in w[:, c])
+        assert Fraction(float(sal[c])) == exact, c
+    # the order column (statistic 1): rows 0..63 = 2^53, 1 x 63; rows 64..127 = 1
+    w2 = np.ones((n, 3))
+    w2[0, 1] = -(2.0 ** 53)                      # |w| is summed: the sign must not matter
+    act2 = np.ones(3, dtype=np.float32)
+    got = O.channel_saliency(w2, act2)
+    assert got[1] == 2.0 ** 53 + 64
+    assert got[0] == got[2] == 128.0
+    ones_first = 0.0
+    for v in sorted(np.abs(w2[:, 1])):          # the other order: the 127 ones, then 2^53
+        ones_first += float(v)
+    assert ones_first == 2.0 ** 53 + 128 != got[1]
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_salient_selection_brute_force_random(seed):
     rng = np.random.default_rng(100 + seed)
