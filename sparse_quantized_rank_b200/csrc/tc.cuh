@@ -111,15 +111,6 @@ CQL_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x
       : "memory");
 }
 
-// 1-D bulk copy global -> shared, completion counted on an mbarrier (both
-// addresses 16-byte aligned, size a multiple of 16).
-CQL_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem]^T with A 2:4 sparse (compressed, M x K/2 in
 // tensor memory) and its selector metadata in tensor memory; kind::f16.
 CQL_DEV void tc_mma_sp_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t meta_tmem, uint32_t idesc,
@@ -129,17 +120,6 @@ CQL_DEV void tc_mma_sp_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uin
       "setp.ne.b32 p, %5, 0;\n\t"
       "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], [%1], %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(meta_tmem), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same with A (compressed) in shared memory, described by a_desc.
-CQL_DEV void tc_mma_sp_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t meta_tmem, uint32_t idesc,
-                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(meta_tmem), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -154,18 +134,10 @@ CQL_DEV void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
-CQL_DEV void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b) : "memory");
-}
 CQL_DEV void tmem_st8(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e, uint32_t f,
                       uint32_t g, uint32_t h) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(a),
                "r"(b), "r"(c), "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
-               : "memory");
-}
-CQL_DEV void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
                : "memory");
 }
 CQL_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
