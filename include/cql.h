@@ -43,9 +43,9 @@
  * ------------------------------------------------------------------------
  * PACKED FORMAT (version 2)
  * ------------------------------------------------------------------------
- * A packed weight is one contiguous device buffer: a 512-byte header followed
- * by up to 13 planes, in the order of the CQL_PLANE_* indices.  Every plane
- * starts on a 256-byte boundary; an absent plane has length 0 and the offset
+ * A packed weight is one contiguous device buffer: a 512-byte header (plane
+ * 0) followed by up to 12 planes (CQL_PLANE_* indices 1-12, in that order).
+ * Every plane starts on a 256-byte boundary; an absent plane has length 0 and the offset
  * where it would start.  All multi-byte fields are little-endian.
  *
  * Header: "CQL1", uint32 version = 2, cql_desc (64 bytes), then the
