@@ -240,3 +240,42 @@ def test_saved_buffer_corruption_is_reported(lib):
     assert status(bad) == C.CQL_ERR_FORMAT
     bad = bytearray(buf); bad[88 + 8 * 13 + 8] ^= 1       # a stored plane length
     assert status(bad) == C.CQL_ERR_FORMAT
+
+
+def test_layout_matches_oracle_on_random_descriptors(lib):
+    """Property check over many valid descriptors (every mask / codec pair the
+    format allows, ragged shapes, adapter ranks, CSR fractions, SLiM^O
+    fields): the library's layout equals the oracle's, planes are 256-byte
+    aligned, in order and disjoint, and the header's size rule holds."""
+    from hypothesis import given, settings, strategies as st
+
+    @st.composite
+    def descs(draw):
+        codec = draw(st.sampled_from([O.CODEC_INT4, O.CODEC_INT3, O.CODEC_LUT3, O.CODEC_LUT4]))
+        lut = codec in (O.CODEC_LUT3, O.CODEC_LUT4)
+        mask = O.MASK_NONE if lut else draw(st.sampled_from([O.MASK_NONE, O.MASK_2_4, O.MASK_BITMAP50]))
+        n = 128 * draw(st.integers(1, 96))
+        k = 128 * draw(st.integers(1, 128 if lut else 512))
+        rank = 16 * draw(st.integers(0, 16))
+        frac = draw(st.sampled_from([0.0, 0.0005, 0.002, 0.0045, 0.0625]))
+        m = draw(st.integers(0, k // 8))
+        e = draw(st.integers(1, 8)) if m else 0
+        return dict(n_out=n, k_in=k, mask=mask, codec=codec, rank=rank, outlier_frac=frac,
+                    salient_channels=m, salient_log2=e)
+
+    @settings(max_examples=400, derandomize=True, deadline=None)
+    @given(descs())
+    def check(kw):
+        lay = C.cql_packed_layout(C.make_desc(**kw))
+        od = O.OracleDesc(kw["n_out"], kw["k_in"], kw["mask"], kw["codec"], 0.9, float(np.float32(kw["outlier_frac"])),
+                          kw["rank"], salient_channels=kw["salient_channels"], salient_log2=kw["salient_log2"])
+        ol = O.packed_layout(od)
+        assert list(lay.off) == ol["off"] and list(lay.len) == ol["len"], kw
+        assert lay.total_bytes == ol["total"] and lay.nnz == ol["nnz"], kw
+        end = 0
+        for i in range(O.NPLANES):
+            assert lay.off[i] % 256 == 0 and lay.off[i] >= end, (kw, i)
+            end = lay.off[i] + lay.len[i]
+        assert lay.len[0] == 512 and lay.total_bytes >= end and lay.total_bytes % 256 == 0
+
+    check()
