@@ -537,6 +537,7 @@ def extra_lines(torch, C, dev, stream, barrier):
         torch.cuda.empty_cache()
     out.append(stack_line(torch, C, dev, stream))
     out.append(adapter_build_line(torch, C, dev, stream))
+    out.extend(pack_lines(torch, C, dev, stream))
     tf_peak, _ = measured_tflops()
     for name in ("prefill_up", "prefill_down"):
         wl = workload(name)
@@ -554,6 +555,57 @@ def extra_lines(torch, C, dev, stream, barrier):
                             "(2:4 codes converted on chip)"})
         del b
         torch.cuda.empty_cache()
+    return out
+
+
+def pack_lines(torch, C, dev, stream, reps=3):
+    """One-time packer cost (pack_compressed_weight) of full-size layers, with
+    and without the packer-side searches: the SLiM-Quant clip search
+    (clip_alpha 0) against a fixed alpha on mlp_up, SqueezeLLM's
+    Fisher-weighted k-means against the plain quantile table on
+    lut_dense_sparse, and the SLiM^O channel selection.  CUDA events around
+    `reps` packs after one warm pack.  A failure is reported in its line
+    instead of ending the run."""
+    from workloads import make_layer_inputs, workload
+    cases = (("mlp_up", {}, "clip alpha fixed (0.9)"),
+             ("mlp_up", {"clip_alpha": 0.0}, "clip alpha searched (SLiM-Quant grid over a |w|/amax histogram)"),
+             ("lut_dense_sparse", {}, "LUT3 centroids from quantiles"),
+             ("lut_dense_sparse", {"fisher": True}, "LUT3 centroids by Fisher-weighted k-means"),
+             ("mlp_up_slimo", {}, "SLiM^O channel selection and scaling"))
+    out = []
+    for name, over, what in cases:
+        wl = workload(name, **over)
+        entry = {"workload": f"pack {wl_name(wl, 1).rsplit(' batch', 1)[0]}", "what": what}
+        try:
+            inp = make_layer_inputs(wl, max_batch=1)
+            W, L, R, _ = device_inputs(torch, inp, wl, dev)
+            act = torch.from_numpy(inp["act_absmean"]).to(dev) if inp["act_absmean"] is not None else None
+            fis = torch.from_numpy(inp["fisher"]).to(dev) if inp["fisher"] is not None else None
+            d = desc_from_workload(C, wl)
+            lay = C.cql_packed_layout(d)
+            packed = torch.empty(lay.total_bytes, dtype=torch.uint8, device=dev)
+            pw = C.cql_pack_workspace_size(d)
+            ws = torch.empty(max(pw, 256), dtype=torch.uint8, device=dev)
+
+            def pack():
+                C.pack_compressed_weight(d, W, C._dt_of(W), L, R, act, fis, packed, lay.total_bytes, ws, pw, stream)
+
+            with torch.cuda.stream(stream):
+                pack()
+                stream.synchronize()
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(stream)
+                for _ in range(reps):
+                    pack()
+                t1.record(stream)
+                stream.synchronize()
+            entry["ms_per_layer"] = round(t0.elapsed_time(t1) / reps, 3)
+            entry["status"] = C.cql_status_string(C.cql_get_device_status(ws, stream))
+            del W, L, R, act, fis, packed, ws
+        except Exception as e:                       # reported, not fatal: the pack is off the timed path
+            entry["error"] = f"{type(e).__name__}: {e}"
+        torch.cuda.empty_cache()
+        out.append(entry)
     return out
 
 
