@@ -241,6 +241,55 @@ def cql_get_device_status(workspace, stream=None) -> int:
 # convenience owner of one packed layer
 # ---------------------------------------------------------------------------
 
+def check_forward_args(desc: cql_desc, x, out=None, device=None) -> None:
+    """Raise ValueError unless x is a contiguous [B][K] fp16/bf16 tensor and
+    out (if given) a contiguous [B][N] fp32/fp16/bf16 tensor, both on
+    ``device`` (the packed layer's).  The C entry point receives raw
+    pointers and cannot see a tensor's size, so a wrong shape would make the
+    kernels read or write past its end: it is refused here."""
+    import torch
+    if x.dim() != 2 or x.shape[1] != desc.k_in or not x.is_contiguous():
+        raise ValueError(f"x must be a contiguous [batch][{desc.k_in}] tensor, got {tuple(x.shape)}")
+    if x.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError(f"x must be float16 or bfloat16, got {x.dtype}")
+    if device is not None and x.device != device:
+        raise ValueError(f"x is on {x.device}, the packed layer on {device}")
+    if out is not None:
+        if tuple(out.shape) != (x.shape[0], desc.n_out) or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous [{x.shape[0]}][{desc.n_out}] tensor, got {tuple(out.shape)}")
+        if out.dtype not in (torch.float32, torch.float16, torch.bfloat16):
+            raise ValueError(f"out must be float32, float16 or bfloat16, got {out.dtype}")
+        if out.device != x.device:
+            raise ValueError(f"out is on {out.device}, x on {x.device}")
+
+
+def check_pack_args(desc: cql_desc, W, L=None, R=None, act_absmean=None, fisher=None) -> None:
+    """Raise ValueError unless the packer's inputs have the shapes and dtypes
+    the descriptor implies (W [N][K] fp32/bf16; L [N][r], R [r][K],
+    act_absmean [K], fisher [N][K] fp32) and share W's device.  The C entry
+    point reads them through raw pointers and cannot check their sizes."""
+    import torch
+    n, k, r = desc.n_out, desc.k_in, desc.rank
+    want = [("W", W, (n, k), (torch.float32, torch.bfloat16))]
+    if r > 0:
+        if L is None or R is None:
+            raise ValueError(f"rank {r} needs L [{n}][{r}] and R [{r}][{k}]")
+        want += [("L", L, (n, r), (torch.float32,)), ("R", R, (r, k), (torch.float32,))]
+    if act_absmean is not None:
+        want.append(("act_absmean", act_absmean, (k,), (torch.float32,)))
+    elif desc.salient_channels > 0:
+        raise ValueError("salient_channels > 0 needs act_absmean [K]")
+    if fisher is not None:
+        want.append(("fisher", fisher, (n, k), (torch.float32,)))
+    for name, t, shape, dts in want:
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        if t.dtype not in dts:
+            raise ValueError(f"{name} must be one of {dts}, got {t.dtype}")
+        if t.device != W.device:
+            raise ValueError(f"{name} is on {t.device}, W on {W.device}")
+
+
 def _dt_of(t) -> int:
     import torch
     return {torch.float32: CQL_DT_F32, torch.float16: CQL_DT_F16, torch.bfloat16: CQL_DT_BF16}[t.dtype]
@@ -259,17 +308,24 @@ class CompressedLinear:
 
     def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None, act_absmean=None, fisher=None):
         import torch
+        check_pack_args(desc, W, L, R, act_absmean, fisher)
         self.desc = desc
         self.layout = cql_packed_layout(desc)
         dev = W.device
         self.packed = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=dev)
         pw = cql_pack_workspace_size(desc)
         pws = torch.empty(max(pw, 256), dtype=torch.uint8, device=dev)
-        pack_compressed_weight(desc, W.contiguous(), _dt_of(W), None if L is None else L.contiguous(),
-                               None if R is None else R.contiguous(),
-                               None if act_absmean is None else act_absmean.contiguous(),
-                               None if fisher is None else fisher.contiguous(), self.packed,
-                               self.layout.total_bytes, pws, pw, stream)
+        args = [None if t is None else t.contiguous() for t in (W, L, R, act_absmean, fisher)]
+        if isinstance(stream, torch.cuda.Stream):
+            # the pack runs on a side stream: keep the allocator from reusing
+            # the inputs' memory (the caller may drop W right away, and the
+            # contiguous copies are temporaries) before that stream is done
+            for t in args:
+                if t is not None:
+                    t.record_stream(stream)
+        Wc, Lc, Rc, ac, fc = args
+        pack_compressed_weight(desc, Wc, _dt_of(Wc), Lc, Rc, ac, fc, self.packed, self.layout.total_bytes, pws, pw,
+                               stream)
         self._pack_ws = pws            # kept alive until the pack kernels ran
         self._ws = {}
 
@@ -312,7 +368,7 @@ class CompressedLinear:
 
     def forward(self, x, out_dtype=None, out=None, flags: Optional[int] = None, stream=None):
         import torch
-        assert x.dim() == 2 and x.shape[1] == self.desc.k_in and x.is_contiguous()
+        check_forward_args(self.desc, x, out, self.packed.device)
         batch = x.shape[0]
         if out is None:
             out = torch.empty(batch, self.desc.n_out, dtype=out_dtype or x.dtype, device=x.device)

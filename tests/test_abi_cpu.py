@@ -279,3 +279,49 @@ def test_layout_matches_oracle_on_random_descriptors(lib):
         assert lay.len[0] == 512 and lay.total_bytes >= end and lay.total_bytes % 256 == 0
 
     check()
+
+
+def test_binding_refuses_mis_shaped_tensors():
+    """The C entry point sees raw pointers only, so the binding checks the
+    tensors' shapes, dtypes, layout and devices before calling it."""
+    import torch
+    d = C.make_desc(256, 512)
+    x = torch.zeros(3, 512, dtype=torch.bfloat16)
+    C.check_forward_args(d, x, torch.zeros(3, 256), torch.device("cpu"))      # valid
+    C.check_forward_args(d, x.half(), None, None)
+    bad = [
+        (torch.zeros(3, 384, dtype=torch.bfloat16), None),                         # K mismatch
+        (torch.zeros(512, 3, dtype=torch.bfloat16).t(), None),                     # not contiguous
+        (torch.zeros(3, 512), None),                                                # fp32 activations
+        (x, torch.zeros(2, 256)),                                                   # out rows
+        (x, torch.zeros(3, 128)),                                                   # out columns
+        (x, torch.zeros(256, 3).t()),                                               # out not contiguous
+        (x, torch.zeros(3, 256, dtype=torch.int32)),                                # out dtype
+    ]
+    for xi, oi in bad:
+        with pytest.raises(ValueError):
+            C.check_forward_args(d, xi, oi, torch.device("cpu"))
+    with pytest.raises(ValueError):                                                 # another device
+        C.check_forward_args(d, x, None, torch.device("cuda", 0))
+
+
+def test_binding_refuses_mis_shaped_pack_inputs():
+    import torch
+    d = C.make_desc(256, 512, rank=16, salient_channels=4, salient_log2=1)
+    W = torch.zeros(256, 512, dtype=torch.bfloat16)
+    L, R, a = torch.zeros(256, 16), torch.zeros(16, 512), torch.ones(512)
+    C.check_pack_args(d, W, L, R, a)                                            # valid
+    C.check_pack_args(C.make_desc(256, 512), W.float())                         # rank 0, no SLiM^O
+    bad = [
+        (W[:128], L, R, a, None),                                               # W rows
+        (W.half(), L, R, a, None),                                              # W dtype
+        (W, None, R, a, None),                                                  # rank needs L
+        (W, L.t().contiguous(), R, a, None),                                    # L transposed
+        (W, L, R.double(), a, None),                                            # R dtype
+        (W, L, R, None, None),                                                  # SLiM^O needs the statistic
+        (W, L, R, torch.ones(256), None),                                       # statistic length
+        (W, L, R, a, torch.ones(512, 256)),                                     # Fisher shape
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            C.check_pack_args(d, *args)
