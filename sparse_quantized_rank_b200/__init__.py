@@ -303,8 +303,11 @@ class CompressedLinear:
     tensor [K] of per-channel mean |x| (SLiM^O layers only), ``fisher`` a
     fp32 CUDA tensor [N][K] Fisher diagonal (LUT codecs: weighted k-means).
     A descriptor with clip_alpha 0 has the packer search alpha; the chosen
-    value is in ``clip_alpha()``.  Buffers are torch tensors allocated once;
-    forward calls allocate only the output tensor (or write into ``out``)."""
+    value is in ``clip_alpha()``.  Buffers are torch tensors: the packed
+    layer once, and one forward workspace per distinct batch size, on the
+    first call at that size (its layout depends on the batch, and the
+    kernels leave it ready for the next call at the same size); later calls
+    allocate only the output tensor (or none, given ``out``)."""
 
     def __init__(self, desc: cql_desc, W, L=None, R=None, stream=None, act_absmean=None, fisher=None):
         import torch
