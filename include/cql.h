@@ -45,8 +45,9 @@
  * ------------------------------------------------------------------------
  * A packed weight is one contiguous device buffer: a 512-byte header (plane
  * 0) followed by up to 12 planes (CQL_PLANE_* indices 1-12, in that order).
- * Every plane starts on a 256-byte boundary; an absent plane has length 0 and the offset
- * where it would start.  All multi-byte fields are little-endian.
+ * Every plane starts on a 256-byte boundary; an absent plane has length 0
+ * and the offset where it would start.  All multi-byte fields are
+ * little-endian.
  *
  * Header: "CQL1", uint32 version = 2, cql_desc (64 bytes), then the
  * cql_layout (uint64 total_bytes, uint64 nnz, uint64 off[13], uint64 len[13]);
@@ -358,7 +359,7 @@ cql_status compressed_linear_forward(const cql_desc* desc, const void* packed, c
  *   (cql_workspace_size) would exceed 4 MiB returns CQL_ERR_SIZE without
  *   launching anything.  The library never calls cudaMalloc or cudaFree here.
  *   The first call on a device finds the array's address and clears it (with
- *   that device current; make this first call before any stream capture).
+ *   that device current).
  *   All calls share the array, and each call first clears (memset on its
  *   stream) the part of it that it uses: calls that overlap on the GPU race,
  *   so order them on one stream.  Device errors are recorded in the array's

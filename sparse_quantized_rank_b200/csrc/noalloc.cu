@@ -10,9 +10,9 @@
 // which every GPU that loads the library holds until the process exits.
 //
 // Set-up: the first call on a device looks up the array's device address with
-// cudaGetSymbolAddress (with that device current) and clears the array; that
-// first call should come before any stream capture.  Every call then shares
-// the same array and clears, on its stream, the part it is about to use.
+// cudaGetSymbolAddress (with that device current) and clears the array.
+// Every call then shares the same array and clears, on its stream, the part
+// it is about to use.
 // Calls whose work overlaps on the GPU (different streams, or different host
 // threads without ordering) race on the array and must be avoided.
 #include <mutex>
