@@ -432,6 +432,11 @@ def _brute_forward(parts, desc, x):
     ("down_unstructured", dict(n=128, k=256, rank=32, codec="int3")),
     ("lut_dense_sparse", dict(n=128, k=256)),
     ("mlp_up_slimo", dict(n=128, k=256, rank=16, salient_channels=4, salient_log2=2)),
+    # the remaining codec / mask / outlier combinations the format allows
+    ("lut_dense_sparse", dict(n=128, k=256, codec="lut4", rank=16)),
+    ("mlp_up", dict(n=128, k=256, codec="int3", outlier_frac=0.01, rank=0)),          # 2:4 int3 + CSR
+    ("down_unstructured", dict(n=128, k=256, codec="int4", outlier_frac=0.0625, rank=16)),  # largest CSR share
+    ("mlp_up", dict(n=128, k=256, mask="none", outlier_frac=0.003, rank=16, clip_alpha=0.0)),
 ])
 def test_forward_matches_brute_force(name, over):
     wl = workload(name, **over)
